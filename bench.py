@@ -1,0 +1,511 @@
+"""Benchmark of the weight-only block-32 qgemv/qgemm path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Default workload ("decoder_block_m1"): one Qwen3-0.6B-style decoder block at decode, M = 1,
+int4 block-32 weights: the 7 projections q[2048x1024], k[1024x1024], v[1024x1024],
+o[1024x2048], gate/up[3072x1024], down[1024x3072]. One step runs the 7 qgemv calls of one
+block; consecutive steps walk the 28 blocks of a seeded synthetic decoder (247.7 MB of
+packed weights, more than the 126 MB L2), so every step streams its weights from HBM.
+Metric: weight GB/s (packed codes + scales per step / time).
+
+Timed region: K steps replayed from CUDA graphs on one stream, bracketed by a barrier and
+device synchronisation, timed with CUDA events on that stream; the max over ranks is
+reported. Under torchrun every rank runs its own replica (no data-path collective).
+
+Also on the JSON line: `e2e` (the same steps through the public API with x copied from
+pinned host memory and y read back every step), `roofline` (the qgemv kernel against the
+measured HBM copy bandwidth), `cpu_baseline` (the CPU oracle on the host cores, a bounded
+sample), `parity` (GPU vs oracle on the sampled step), and `prefill` (the tcgen05 qgemm over
+all 7 projections of all 28 blocks at M = 512, TFLOP/s against the measured bf16 peak).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from weight_only_bit_qgemv_b200 import workloads  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# --------------------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, ms_per_rank: float, world: int):
+    """(whole-job units/s, max ms) with the max-over-ranks time as the job's time."""
+    ms = max_over_ranks(ms_per_rank, world)
+    return units_per_rank * world / (ms / 1e3), ms
+
+
+# --------------------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        time.sleep(0.25)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------------
+# the workload
+# --------------------------------------------------------------------------------------
+
+def build_decoder(bits: int, device, n_layers: int = workloads.N_LAYERS):
+    import weight_only_bit_qgemv_b200 as woq
+
+    layers = []
+    for layer in range(n_layers):
+        projs = []
+        for p, (_, n, k) in enumerate(workloads.DECODER_PROJ):
+            W = workloads.weight(n, k, seed=workloads.layer_seed(layer, p))
+            projs.append(woq.pack(W, bits, device))
+        layers.append(projs)
+    return layers
+
+
+def decode_step_bytes(layer):
+    return sum(w.nbytes for w in layer)
+
+
+def time_graph_steps(step_fn, n_cycle: int, steps: int, warmup: int, stream, world):
+    """Capture step_fn(i) for i in [0, n_cycle) into a graph; replay to cover `steps` steps.
+
+    Returns (ms for the K timed steps, launches of our kernels per step).
+    """
+    import weight_only_bit_qgemv_b200 as woq
+
+    def capture(count, start):
+        g = torch.cuda.CUDAGraph()
+        c0 = woq.launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(count):
+                step_fn((start + i) % n_cycle)
+        return g, woq.launch_count() - c0
+
+    with torch.cuda.stream(stream):
+        for i in range(min(2, n_cycle)):  # eager warm-up (allocations, attribute setup)
+            step_fn(i)
+    stream.synchronize()
+    full, launches_full = capture(n_cycle, 0)
+    rem = steps % n_cycle
+    g_rem = capture(rem, 0)[0] if rem else None
+    per_step = launches_full / n_cycle
+
+    # warm-up steps, untimed
+    w_full, w_rem = divmod(warmup, n_cycle)
+    g_wrem = capture(w_rem, 0)[0] if w_rem else None
+    with torch.cuda.stream(stream):
+        for _ in range(w_full):
+            full.replay()
+        if g_wrem is not None:
+            g_wrem.replay()
+    stream.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps // n_cycle):
+            full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end), per_step
+
+
+def run_decode(args, world, rank, local, peaks, peak_kind):
+    import weight_only_bit_qgemv_b200 as woq
+
+    device = torch.device("cuda", local)
+    bits = 4
+    layers = build_decoder(bits, device)
+    xs = [workloads.activations(1, k, seed=workloads.X_SEED + p).to(device)
+          for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
+    ys = [torch.empty(1, n, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    step_bytes = decode_step_bytes(layers[0])
+    total_bytes = sum(decode_step_bytes(l) for l in layers)
+
+    def step(i):
+        for p, w in enumerate(layers[i]):
+            woq.qgemv(xs[p], w, out=ys[p])
+
+    stream = torch.cuda.Stream(device)
+    with ClockSampler(local) as clk:
+        ms, per_step = time_graph_steps(step, len(layers), args.steps, args.warmup, stream, world)
+    clocks = clk.summary()
+    value, ms_max = aggregate_throughput(step_bytes * args.steps, ms, world)
+    gbs = value / 1e9
+
+    # the qgemv kernel against the HBM roofline: every launch in the timed region is it
+    launches = per_step * args.steps
+    achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "peak_source": peak_kind,
+                "bytes_per_launch": round(step_bytes / per_step),
+                "avg_launch_us": round(ms * 1e3 / launches, 3)}
+
+    e2e = run_decode_e2e(layers, device, min(args.steps, 2000), stream, world)
+
+    out = {
+        "metric": "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)",
+        "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "decoder_block_m1", "bits": 4, "block": 32, "m": 1,
+                   "projections": [f"{nm}[{n}x{k}]" for nm, n, k in workloads.DECODER_PROJ],
+                   "layers_cycled": len(layers), "weight_bytes_per_step": step_bytes,
+                   "l2": f"inputs larger than L2: steps walk {len(layers)} blocks, "
+                         f"{total_bytes / 1e6:.1f} MB of packed weights > 126 MB L2",
+                   "launch": "CUDA graph of qgemv C-ABI calls, programmatic dependent launch",
+                   "parallelism": f"replicas x{world}"},
+        "hbm_frac": round(gbs / world / peaks["hbm_gbs"], 4),
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "roofline": roofline,
+    }
+    return out, layers, xs, ys
+
+
+def run_decode_e2e(layers, device, steps, stream, world):
+    """Same steps through the public API, x from pinned host memory, y read back each step."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    host_x = [workloads.activations(1, k, seed=workloads.X_SEED + p).pin_memory()
+              for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
+    host_y = [torch.empty(1, n).pin_memory() for (_, n, k) in workloads.DECODER_PROJ]
+    dx = [torch.empty(1, k, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    dy = [torch.empty(1, n, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    h2d = sum(t.numel() * 4 for t in host_x)
+    d2h = sum(t.numel() * 4 for t in host_y)
+
+    def step(i):
+        for p, w in enumerate(layers[i % len(layers)]):
+            dx[p].copy_(host_x[p], non_blocking=True)
+            woq.qgemv(dx[p], w, out=dy[p])
+            host_y[p].copy_(dy[p], non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(5):
+            step(i)
+        barrier(world)
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(steps):
+            step(i)
+        end.record(stream)
+        end.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    value, _ = aggregate_throughput(decode_step_bytes(layers[0]) * steps, ms, world)
+    return {"value": round(value / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps}
+
+
+def run_prefill(layers, device, m: int, reps: int, peaks, peak_kind, world):
+    """tcgen05 qgemm through all 7 projections of all blocks at M = m (one pass = one rep)."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    Xs = [workloads.activations(m, k, seed=workloads.X_SEED + p).to(device)
+          for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
+    Ys = [torch.empty(m, n, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    ws = torch.empty(max(woq.qgemm_workspace_bytes(m, w, "bf16_tc") for w in layers[0]),
+                     dtype=torch.uint8, device=device)
+    flops = 2.0 * m * sum(n * k for _, n, k in workloads.DECODER_PROJ) * len(layers)
+
+    def step(i):
+        for layer in layers:
+            for p, w in enumerate(layer):
+                woq.qgemm(Xs[p], w, path="bf16_tc", out=Ys[p], workspace=ws)
+
+    stream = torch.cuda.Stream(device)
+    ms, per_step = time_graph_steps(step, 1, reps, 2, stream, world)
+    tflops = flops * reps / (ms / 1e3) / 1e12
+    return {"workload": f"prefill_m{m}", "m": m, "gemms_per_pass": len(layers) * 7,
+            "flop_per_pass": flops, "passes": reps, "ms_per_pass": ms / reps,
+            "tflops": round(tflops, 1), "peak_tflops": peaks["bf16_tflops"],
+            "frac": round(tflops / peaks["bf16_tflops"], 4), "peak_source": peak_kind,
+            "launches_per_pass": int(per_step)}
+
+
+# --------------------------------------------------------------------------------------
+# CPU oracle (cpu_baseline leg and the reference arm)
+# --------------------------------------------------------------------------------------
+
+def oracle_decode_pass(packed_layer, xs_np, rows=None):
+    """One decode step of a block through the oracle; ``rows`` limits each projection."""
+    import oracle
+
+    outs = []
+    for p, (pk, sc, bits) in enumerate(packed_layer):
+        if rows is not None:
+            pk, sc = pk[:rows[p]], sc[:rows[p]]
+        outs.append(oracle.qgemv_ref(xs_np[p], pk, sc, bits))
+    return outs
+
+
+def oracle_layer_inputs(bits=4, layer=0):
+    """Packed weights of one block, quantised and packed by the oracle itself, and x rows."""
+    import oracle
+
+    out = []
+    for p, (_, n, k) in enumerate(workloads.DECODER_PROJ):
+        W = workloads.weight(n, k, seed=workloads.layer_seed(layer, p)).numpy()
+        q, s = oracle.quantise(W, bits)
+        out.append((oracle.pack(q, bits), s, bits))
+    xs = [workloads.activations(1, k, seed=workloads.X_SEED + p).numpy()
+          for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
+    return out, xs
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(packed_layer, xs, budget_s: float):
+    """Median seconds per decode-block pass of the oracle; the outputs of the last pass."""
+    oracle_decode_pass(packed_layer, xs)  # discarded warm-up
+    times, outs = [], None
+    t_end = time.perf_counter() + budget_s
+    while len(times) < 3 or time.perf_counter() < t_end:
+        t0 = time.perf_counter()
+        outs = oracle_decode_pass(packed_layer, xs)
+        times.append(time.perf_counter() - t0)
+        if len(times) >= 50:
+            break
+    return statistics.median(times), len(times), outs
+
+
+def cpu_baseline_leg(layer0_gpu, xs_gpu, budget_s):
+    import weight_only_bit_qgemv_b200 as woq
+
+    packed, xs = oracle_layer_inputs()
+    sec, passes, outs = time_oracle(packed, xs, budget_s)
+    nbytes = sum(pk.nbytes + sc.nbytes for pk, sc, _ in packed)
+    # parity of the GPU step against the oracle on the same inputs (block 0)
+    errs = []
+    for p, w in enumerate(layer0_gpu):
+        y = woq.qgemv(xs_gpu[p], w).cpu().numpy()
+        ref = outs[p]
+        errs.append(float(np.max(np.abs(y - ref)) / np.max(np.abs(ref))))
+    return ({"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+             "kind": "oracle",
+             "sample": f"{passes} passes of decoder block 0 (7 projections, M=1, int4) through the "
+                       f"NumPy float64 oracle, median pass {sec * 1e3:.1f} ms"},
+            {"max_rel_err": max(errs), "tolerance": 1e-4, "checked": "block 0, all 7 outputs"})
+
+
+def run_reference(args, world, rank, budget_s=90.0):
+    """The oracle as it stands, on the host cores, same metric and config (rank 0 only).
+
+    Each of the K (+W) steps is a bounded sample of the decode step: the first rows of each
+    of the 7 projections, sized from one untimed full pass so the whole run takes about
+    ``budget_s`` seconds.
+    """
+    if rank != 0:
+        return None
+    packed, xs = oracle_layer_inputs()
+    t0 = time.perf_counter()
+    oracle_decode_pass(packed, xs)
+    full = time.perf_counter() - t0
+    frac = min(1.0, budget_s / (args.steps + args.warmup) / full)
+    rows = [max(1, int(round(frac * n))) for (_, n, k) in workloads.DECODER_PROJ]
+    nbytes = sum(r * (pk.shape[1] + 2 * sc.shape[1]) for r, (pk, sc, _) in zip(rows, packed))
+    for _ in range(args.warmup):
+        oracle_decode_pass(packed, xs, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_decode_pass(packed, xs, rows)
+    sec = time.perf_counter() - t0
+    value = nbytes * args.steps / sec / 1e9
+    sample = (f"each step: rows {rows} of the 7 projections of decoder block 0 (M=1, int4), "
+              f"{nbytes} weight bytes, through the NumPy float64 oracle; one full block pass "
+              f"took {full * 1e3:.0f} ms")
+    return {"impl": "reference",
+            "metric": "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)",
+            "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "decoder_block_m1", "bits": 4, "block": 32, "m": 1},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=28000)
+    ap.add_argument("--warmup", type=int, default=280)
+    ap.add_argument("--impl", default="woq", choices=["woq", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-m", type=int, default=512)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    peaks, peak_kind = load_peaks()
+    out, layers, xs, ys = run_decode(args, world, rank, local, peaks, peak_kind)
+    if not args.no_prefill:
+        out["prefill"] = run_prefill(layers, torch.device("cuda", local), args.prefill_m, 3,
+                                     peaks, peak_kind, world)
+    if rank == 0 and world >= 1 and not args.no_cpu_baseline:
+        cb, parity = cpu_baseline_leg(layers[0], xs, args.cpu_budget)
+        out["cpu_baseline"] = cb
+        out["parity"] = parity
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,169 @@
+/*
+ * woq.h -- C ABI of libwoq: weight-only block-32 int4/int8 quantised matmul on B200 (sm_100a).
+ *
+ * What is computed. Weights W [n, k] (out, in) are stored packed as symmetric signed
+ * integers in blocks of 32 consecutive values along k, one IEEE binary16 scale per block;
+ * activations and results are FP32 and the products accumulate in FP32; dequantisation is
+ * fused into the multiply and no dequantised weight tensor is ever written. The pages
+ * this follows:
+ *   - "TinyMOSS-Diarize" (devpost), "How we built it": strictly weight-only kernels, FP32
+ *     activations, dequantisation fused into the matmul, no materialised dequantised
+ *     weights; a blocked GEMM path for prefill and a separate GEMV path for decode; packed
+ *     tensors in a container whose tensor table is 64-byte aligned.
+ *   - "MOSS-Transcribe-Diarize -- LiteRT (TFLite)", "Files": the production decoder is
+ *     int4 in blocks of 32 ("q4b32").
+ *   - "MOSS Transcribe Diarize 0.9B" (soniqo, Russian guide), "Implementation notes":
+ *     symmetric linear INT8 quantisation with block 32 for the decoder.
+ *
+ * Packed layout (fixed; qpack produces it bit-exactly):
+ *   bits == 4: row r of W occupies k/2 bytes at packed + r*k/2. Byte j holds element 2j in
+ *              bits 0-3 and element 2j+1 in bits 4-7, each a 4-bit two's-complement code
+ *              in [-8, 7].
+ *   bits == 8: row r occupies k bytes at packed + r*k, one two's-complement byte per
+ *              element, codes in [-128, 127].
+ *   scales:    binary16 bit patterns, [n, k/32] row-major; element (r, j) scales codes
+ *              k in [32j, 32j+32) of row r. W_hat[r, c] = scale[r, c/32] * code[r, c].
+ *   All codes a container may hold are decoded, including -8 / -128, which qpack never
+ *   emits.
+ *
+ * Conventions for every call:
+ *   - Return WOQ_OK (0) or a negative WOQ_E* status; arguments are checked before any
+ *     work is queued, and a failed check queues nothing.
+ *   - Device pointers are CUDA device addresses on the current device; the caller owns
+ *     every buffer and the stream. The library allocates no memory and never
+ *     synchronises the stream; results are ready when the caller's stream reaches them.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   - Kernel faults, if any, surface at the caller's next synchronisation.
+ */
+#ifndef WOQ_H
+#define WOQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define WOQ_OK          0
+#define WOQ_EINVAL     -1  /* null pointer, bits not 4/8, block not 32, m out of range, bad path */
+#define WOQ_ESHAPE     -2  /* n or k <= 0, k % 32 != 0, or a size above a documented limit    */
+#define WOQ_EALIGN     -3  /* packed/scales not 64-byte aligned, or x/y not 16-byte aligned    */
+#define WOQ_ERANGE     -4  /* qpack: non-finite weight, or a block scale overflows binary16    */
+#define WOQ_EDEVICE    -5  /* the current device is not compute capability 10.0 (B200)        */
+#define WOQ_ECUDA      -6  /* a CUDA runtime call or kernel launch failed                     */
+#define WOQ_ETIMEOUT   -7  /* a bounded device-side wait gave up (see woq_device_status)      */
+#define WOQ_EWORKSPACE -8  /* qgemm: workspace null or smaller than qgemm_workspace_bytes     */
+
+/* qgemm paths. */
+#define WOQ_PATH_AUTO     0  /* BF16_TC when m >= 128 (see qgemm), FP32 otherwise          */
+#define WOQ_PATH_FP32     1  /* FP32 products and accumulation (CUDA cores), exact codes      */
+#define WOQ_PATH_BF16_TC  2  /* tcgen05 tensor cores on bf16(X) and bf16(scale*code)          */
+
+/*
+ * One packed weight [n, k] in device memory.
+ *   bits    4 or 8
+ *   block   must be 32
+ *   n, k    rows (out features) and columns (in features); k % 32 == 0
+ *   packed  device pointer, 64-byte aligned, n*k*bits/8 bytes in the layout above
+ *   scales  device pointer, 64-byte aligned, n*(k/32) binary16 bit patterns
+ */
+typedef struct woq_weight {
+  int32_t bits;
+  int32_t block;
+  int64_t n;
+  int64_t k;
+  const uint8_t *packed;
+  const uint16_t *scales;
+} woq_weight;
+
+/*
+ * qpack -- host-side quantiser (all pointers are HOST memory; no GPU is used).
+ * Follows the formats of "MOSS-Transcribe-Diarize -- LiteRT (TFLite)", "Files" (q4b32) and
+ * the soniqo Russian guide, "Implementation notes" (symmetric INT8 block-32). For each row
+ * r and block j:
+ *   a = max |W[r, 32j .. 32j+31]|                                  (exact, over the floats)
+ *   s = binary16 round-half-even of (double)a / qmax, qmax = 7 (int4) or 127 (int8)
+ *   q = clamp(round-half-even((double)w / (double)s), -2^(bits-1), 2^(bits-1)-1), or 0 if s == 0
+ * and writes q into `packed` and the bit pattern of s into `scales`, in the layout above.
+ *   W       [n, k] float32, row-major
+ *   packed  out, n*k*bits/8 bytes;  scales  out, n*(k/32) uint16
+ * Errors: WOQ_EINVAL (null pointer, bits), WOQ_ESHAPE (n, k), WOQ_ERANGE (a non-finite W,
+ * or a scale that rounds to infinity: a/qmax >= 65520). On error the outputs may be
+ * partially written.
+ */
+int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, uint16_t *scales);
+
+/*
+ * qgemv -- decode path, y[m, n] = x[m, k] . W_hat^T for 1 <= m <= 64 ("TinyMOSS-Diarize",
+ * "How we built it": the separate GEMV path for decode). FP32 products and accumulation
+ * (CUDA cores); within a 32-block the codes are multiplied exactly and the block sum is
+ * scaled once. Deterministic: the same inputs give the same bits on every call.
+ *   x  device, [m, k] float32 row-major, 16-byte aligned
+ *   w  host pointer to the weight descriptor (read during the call only)
+ *   y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
+ * Limits: k <= 32768 (the x rows are staged in shared memory). Errors: WOQ_EINVAL,
+ * WOQ_ESHAPE, WOQ_EALIGN, WOQ_EDEVICE, WOQ_ECUDA.
+ */
+int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream);
+
+/*
+ * Bytes of device workspace qgemm needs for (m, w, path); 0 if none. Returns 0 for
+ * invalid arguments too (qgemm itself reports those).
+ */
+size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path);
+
+/*
+ * qgemm -- prefill path, Y[m, n] = X[m, k] . W_hat^T for any m >= 1 ("TinyMOSS-Diarize",
+ * "How we built it": the blocked GEMM path for prefill, each weight tile unpacked once
+ * and reused across activation rows).
+ *   path WOQ_PATH_BF16_TC: X is rounded to bf16 into the workspace, each weight tile is
+ *        dequantised once into shared memory as bf16(scale*code) and multiplied on the
+ *        tcgen05 tensor cores with FP32 accumulation in tensor memory.
+ *   path WOQ_PATH_FP32: the same FP32 arithmetic as qgemv, for any m.
+ *   path WOQ_PATH_AUTO: BF16_TC if m >= 128, else FP32.
+ *   X  device, [m, k] float32 row-major, 16-byte aligned
+ *   Y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
+ *   workspace  device, 256-byte aligned, at least qgemm_workspace_bytes(m, w, path) bytes
+ *              (may be NULL when that is 0); its contents on entry do not matter, and
+ *              calls sharing one workspace must be ordered on one stream
+ * Errors: WOQ_EINVAL, WOQ_ESHAPE, WOQ_EALIGN, WOQ_EDEVICE, WOQ_EWORKSPACE, WOQ_ECUDA.
+ * If a bounded wait gives up inside the tensor-core kernel, the kernel records the event,
+ * drains its in-flight copies and MMAs, frees its tensor memory and returns, leaving Y
+ * unspecified; woq_device_status reports it.
+ */
+int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path,
+          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * woq_device_status -- synchronises the current device, then returns WOQ_ETIMEOUT if any
+ * kernel of this library recorded a bounded wait that gave up since the last call with
+ * clear != 0 (and clears the record if clear != 0), WOQ_ECUDA if synchronisation failed,
+ * else WOQ_OK.
+ */
+int woq_device_status(int clear);
+
+/*
+ * woq_debug_set_wait_limit -- test hook. Sets the cycle budget of every bounded wait in the
+ * tensor-core qgemm kernel for launches that follow: cycles > 0 sets it, cycles < 0 makes
+ * every wait that would have to spin give up at once (so the timeout path can be exercised
+ * without a hang), 0 restores the default (2^32 cycles, about two seconds). Host-side state
+ * of the process, not thread-safe against concurrent launches.
+ */
+void woq_debug_set_wait_limit(long long cycles);
+
+/* Human-readable text for a status code (static storage; never NULL). */
+const char *woq_status_str(int status);
+
+/* Number of kernels this library has launched in this process (all devices). */
+uint64_t woq_launch_count(void);
+
+/* ABI version of this header: 1. */
+int woq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WOQ_H */

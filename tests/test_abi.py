@@ -1,0 +1,89 @@
+"""The C-ABI library loads and exports every symbol include/woq.h declares (CPU only).
+
+Only calls that return before touching a device are made here: argument checks and
+workspace sizing. Compute is exercised by the gpu-marked tests.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_only_bit_qgemv_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "woq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b(\w+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = _lib.lib()
+    declared = _declared()
+    assert "qpack" in declared and "qgemv" in declared and "qgemm" in declared
+    assert sorted(_lib.EXPORTS) == declared
+    for name in declared:
+        assert hasattr(L, name), name
+    assert L.woq_abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(0, -9, -1):
+        s = _lib.status_str(code)
+        assert s and s != "unknown status"
+    assert _lib.status_str(-99) == "unknown status"
+
+
+def _w(bits=4, n=64, k=64, packed=64, scales=128, block=32):
+    return _lib.WoqWeight(bits, block, n, k, packed, scales)
+
+
+def test_argument_checks_return_before_touching_a_device():
+    L = _lib.lib()
+    ok_ptr = 1 << 20  # never dereferenced: every call below fails validation first
+    cases = [
+        (_w(bits=5), _lib.WOQ_EINVAL),
+        (_w(block=16), _lib.WOQ_EINVAL),
+        (_w(k=48), _lib.WOQ_ESHAPE),
+        (_w(n=0), _lib.WOQ_ESHAPE),
+        (_w(packed=ok_ptr + 32), _lib.WOQ_EALIGN),
+        (_w(scales=ok_ptr + 2), _lib.WOQ_EALIGN),
+        (_w(packed=0), _lib.WOQ_EINVAL),
+    ]
+    for w, want in cases:
+        assert L.qgemv(ok_ptr, 1, ctypes.byref(w), ok_ptr, None) == want
+        assert L.qgemm(ok_ptr, 1, ctypes.byref(w), ok_ptr, 0, None, 0, None) == want
+    w = _w(packed=ok_ptr, scales=ok_ptr)
+    assert L.qgemv(ok_ptr, 0, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv(ok_ptr, 65, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv(None, 1, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv(ok_ptr + 4, 1, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EALIGN
+    big = _w(k=65536, packed=ok_ptr, scales=ok_ptr)
+    assert L.qgemv(ok_ptr, 1, ctypes.byref(big), ok_ptr, None) == _lib.WOQ_ESHAPE
+    # bf16 path: workspace checked before the device
+    need = L.qgemm_workspace_bytes(256, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC)
+    assert need == 256 * 64 * 2
+    assert L.qgemm(ok_ptr, 256, ctypes.byref(w), ok_ptr, 2, None, 0, None) == _lib.WOQ_EWORKSPACE
+    assert L.qgemm(ok_ptr, 256, ctypes.byref(w), ok_ptr, 2, ok_ptr, need - 1, None) == _lib.WOQ_EWORKSPACE
+    assert L.qgemm(ok_ptr, 256, ctypes.byref(w), ok_ptr, 2, ok_ptr + 16, need, None) == _lib.WOQ_EALIGN
+    assert L.qgemm(ok_ptr, 4, ctypes.byref(w), ok_ptr, 7, None, 0, None) == _lib.WOQ_EINVAL
+
+
+def test_workspace_sizing():
+    L = _lib.lib()
+    w = _w(n=1024, k=3072, packed=1 << 20, scales=1 << 20)
+    assert L.qgemm_workspace_bytes(4, ctypes.byref(w), _lib.WOQ_PATH_FP32) == 0
+    assert L.qgemm_workspace_bytes(4, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 0
+    assert L.qgemm_workspace_bytes(512, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 512 * 3072 * 2
+    assert L.qgemm_workspace_bytes(375, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC) % 256 == 0
+    assert L.qgemm_workspace_bytes(0, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC) == 0
+    assert L.qgemm_workspace_bytes(16, ctypes.byref(_w(bits=3)), 0) == 0
+
+
+def test_launch_counter_starts_readable():
+    assert _lib.lib().woq_launch_count() >= 0

@@ -1,0 +1,135 @@
+"""GPU parity of qgemv (FP32 decode path) against the CPU oracle, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import weight_only_bit_qgemv_b200 as woq
+from weight_only_bit_qgemv_b200 import workloads
+from tests.gpu_util import (FP32_TOL, guarded_out, max_rel, packed_from_weight, packed_raw,
+                            ref_rows, tail_intact)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 7, 8, 16, 33, 64])
+def test_qgemv_all_m(bits, m):
+    n, k = 1000, 2048  # ragged n (not a multiple of any row grouping), two chunks per lane
+    W = workloads.weight(n, k, seed=11 + m)
+    w, p, s = packed_from_weight(W, bits)
+    x = workloads.activations(m, k, seed=100 + m)
+    y = woq.qgemv(x.cuda(), w).cpu().numpy()
+    assert max_rel(y, ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("proj", range(7))
+def test_decoder_block_shapes_m1(bits, proj):
+    name, n, k = workloads.DECODER_PROJ[proj]
+    W = workloads.weight(n, k, seed=workloads.layer_seed(0, proj))
+    w, p, s = packed_from_weight(W, bits)
+    x = workloads.activations(1, k, seed=workloads.X_SEED)
+    y = woq.qgemv(x.cuda(), w).cpu().numpy()
+    assert max_rel(y, ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL, name
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_lm_head_full_size_sampled(bits):
+    n, k = workloads.LM_HEAD
+    W = workloads.weight(n, k, seed=workloads.LM_HEAD_SEED)
+    w, p, s = packed_from_weight(W, bits)
+    x = workloads.activations(1, k, seed=workloads.X_SEED)
+    buf, y = guarded_out(1, n)
+    woq.qgemv(x.cuda(), w, out=y)
+    yc = y.cpu().numpy()
+    assert tail_intact(buf, 1, n)
+    assert np.all(np.isfinite(yc))
+    rows = np.random.default_rng(0).choice(n, 2048, replace=False)
+    rows = np.concatenate([rows, [0, 1, n - 2, n - 1]])
+    assert max_rel(yc[:, rows], ref_rows(x.numpy(), p, s, bits, rows)) <= FP32_TOL
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("m", [1, 5])
+def test_every_code_including_the_negative_extreme(bits, m):
+    n, k = 257, 1024
+    w, p, s = packed_raw(n, k, bits, seed=bits * 10 + m)
+    x = workloads.activations(m, k, seed=3)
+    y = woq.qgemv(x.cuda(), w).cpu().numpy()
+    assert max_rel(y, ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("kind", ["one_hot", "ones", "alternating"])
+def test_adversarial_x(bits, kind):
+    n, k = 512, 1024
+    w, p, s = packed_raw(n, k, bits, seed=77)
+    x = np.zeros((3, k), dtype=np.float32)
+    if kind == "one_hot":
+        x[0, 0] = 1.0
+        x[1, k - 1] = -2.0
+        x[2, 517] = 3.0
+    elif kind == "ones":
+        x[:] = 1.0
+    else:
+        x[:, 0::2] = 1.0
+        x[:, 1::2] = -1.0
+        x[1] *= 1e-3
+        x[2] *= 1e3
+    y = woq.qgemv(torch.from_numpy(x).cuda(), w).cpu().numpy()
+    ref = ref_rows(x, p, s, bits)
+    for r in range(3):  # per x row: each row's own scale
+        assert max_rel(y[r:r + 1], ref[r:r + 1]) <= FP32_TOL
+    if kind == "one_hot":  # a single product per output: exact
+        np.testing.assert_array_equal(y, ref.astype(np.float32))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("n,k", [(1, 32), (31, 96), (33, 64), (129, 160), (4099, 512)])
+def test_small_and_ragged_shapes(bits, n, k):
+    W = workloads.weight(n, k, seed=n + k)
+    w, p, s = packed_from_weight(W, bits)
+    for m in (1, 3, 9):
+        x = workloads.activations(m, k, seed=m)
+        buf, y = guarded_out(m, n)
+        woq.qgemv(x.cuda(), w, out=y)
+        assert tail_intact(buf, m, n)
+        assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL
+
+
+def test_zero_weight_gives_exact_zero():
+    W = torch.zeros(300, 1024)
+    w, _, _ = packed_from_weight(W, 4)
+    y = woq.qgemv(workloads.activations(2, 1024, 1).cuda(), w)
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_identity_closed_form():
+    K = 1024
+    w, _, _ = packed_from_weight(torch.eye(K), 4)
+    x = workloads.activations(1, K, seed=5)
+    y = woq.qgemv(x.cuda(), w).cpu()
+    torch.testing.assert_close(y, x * (1 - 2.0 ** -12), rtol=2e-7, atol=0)
+
+
+def test_deterministic_bits():
+    W = workloads.weight(3072, 1024, seed=1)
+    w, _, _ = packed_from_weight(W, 4)
+    x = workloads.activations(4, 1024, seed=2).cuda()
+    a = woq.qgemv(x, w)
+    b = woq.qgemv(x, w)
+    assert torch.equal(a, b)
+
+
+def test_launches_are_counted_and_stream_ordered():
+    W = workloads.weight(2048, 1024, seed=3)
+    w, p, s = packed_from_weight(W, 8)
+    x = workloads.activations(1, 1024, seed=4)
+    st = torch.cuda.Stream()
+    before = woq.launch_count()
+    with torch.cuda.stream(st):
+        y = woq.qgemv(x.cuda(), w)
+    st.synchronize()
+    assert woq.launch_count() - before == 1
+    assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, 8)) <= FP32_TOL

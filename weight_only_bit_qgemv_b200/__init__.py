@@ -1,0 +1,143 @@
+"""Weight-only block-32 int4/int8 qgemv/qgemm for B200 (sm_100a).
+
+Thin Python binding over libwoq's C ABI (include/woq.h). PyTorch provides device memory
+and streams only; every step of the computation runs in the library's CUDA kernels (or,
+for ``qpack``, in its host C++ quantiser). There is no CPU or PyTorch fallback: if the
+library is missing, every call raises.
+
+    w = pack(W_fp32_cpu, bits=4, device="cuda")    # qpack on the host, copy to HBM
+    y = qgemv(x, w)                                # decode, 1 <= m <= 64, FP32
+    Y = qgemm(X, w, path="bf16_tc")                # prefill, tcgen05 tensor cores
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import WOQ_PATH_AUTO, WOQ_PATH_BF16_TC, WOQ_PATH_FP32, WoqError  # noqa: F401
+
+__all__ = [
+    "PackedWeight",
+    "qpack",
+    "pack",
+    "qgemv",
+    "qgemm",
+    "qgemm_workspace_bytes",
+    "device_status",
+    "launch_count",
+    "WoqError",
+]
+
+_PATHS = {"auto": WOQ_PATH_AUTO, "fp32": WOQ_PATH_FP32, "bf16_tc": WOQ_PATH_BF16_TC}
+
+
+def _ptr(t: torch.Tensor) -> int:
+    return t.data_ptr()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class PackedWeight:
+    """One packed weight in device memory, in the layout of include/woq.h."""
+
+    packed: torch.Tensor  # uint8 [n, k*bits/8]
+    scales: torch.Tensor  # int16 [n, k/32], binary16 bit patterns
+    bits: int
+    n: int
+    k: int
+
+    def desc(self) -> _lib.WoqWeight:
+        return _lib.WoqWeight(self.bits, 32, self.n, self.k, _ptr(self.packed), _ptr(self.scales))
+
+    @property
+    def nbytes(self) -> int:
+        """Packed codes plus scales: the bytes one product streams from memory."""
+        return self.packed.numel() + 2 * self.scales.numel()
+
+    def to(self, device) -> "PackedWeight":
+        return PackedWeight(self.packed.to(device), self.scales.to(device), self.bits, self.n, self.k)
+
+
+def qpack(W: torch.Tensor, bits: int) -> tuple[torch.Tensor, torch.Tensor]:
+    """Host quantiser (C ABI ``qpack``): W float32 [n, k] on the CPU -> (packed, scales)."""
+    if W.device.type != "cpu" or W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("qpack takes a 2-D float32 CPU tensor")
+    W = W.contiguous()
+    n, k = W.shape
+    if bits not in (4, 8) or k % 32:
+        raise ValueError("bits must be 4 or 8 and k a multiple of 32")
+    packed = torch.empty(n, k * bits // 8, dtype=torch.uint8)
+    scales = torch.empty(n, k // 32, dtype=torch.int16)
+    _lib.check(_lib.lib().qpack(_ptr(W), n, k, bits, _ptr(packed), _ptr(scales)), "qpack")
+    return packed, scales
+
+
+def pack(W: torch.Tensor, bits: int, device="cuda") -> PackedWeight:
+    """qpack on the host, then one copy of codes and scales to ``device``."""
+    packed, scales = qpack(W, bits)
+    n, k = W.shape
+    return PackedWeight(packed.to(device), scales.to(device), bits, n, k)
+
+
+def qgemv(x: torch.Tensor, w: PackedWeight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[m, n] = x[m, k] . W_hat^T, 1 <= m <= 64, FP32 (C ABI ``qgemv``)."""
+    if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty(m, w.n, dtype=torch.float32, device=x.device)
+    d = w.desc()
+    _lib.check(_lib.lib().qgemv(_ptr(x), m, ctypes.byref(d), _ptr(out), _stream(stream)), "qgemv")
+    return out
+
+
+def qgemm_workspace_bytes(m: int, w: PackedWeight, path: str = "auto") -> int:
+    d = w.desc()
+    return int(_lib.lib().qgemm_workspace_bytes(m, ctypes.byref(d), _PATHS[path]))
+
+
+def qgemm(
+    X: torch.Tensor,
+    w: PackedWeight,
+    path: str = "auto",
+    out: torch.Tensor | None = None,
+    workspace: torch.Tensor | None = None,
+    stream=None,
+) -> torch.Tensor:
+    """Y[m, n] = X[m, k] . W_hat^T (C ABI ``qgemm``); path in {"auto", "fp32", "bf16_tc"}."""
+    if X.dtype != torch.float32 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous 2-D float32 CUDA tensor")
+    m = X.shape[0]
+    p = _PATHS[path]
+    if out is None:
+        out = torch.empty(m, w.n, dtype=torch.float32, device=X.device)
+    d = w.desc()
+    need = int(_lib.lib().qgemm_workspace_bytes(m, ctypes.byref(d), p))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _lib.check(
+        _lib.lib().qgemm(_ptr(X), m, ctypes.byref(d), _ptr(out), p, ws_ptr, ws_bytes, _stream(stream)),
+        "qgemm",
+    )
+    return out
+
+
+def device_status(clear: bool = True) -> int:
+    """Synchronise the device and report bounded waits that gave up (C ABI woq_device_status)."""
+    return int(_lib.lib().woq_device_status(1 if clear else 0))
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(_lib.lib().woq_launch_count())

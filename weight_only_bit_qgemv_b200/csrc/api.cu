@@ -1,0 +1,144 @@
+// C-ABI entry points of libwoq (declared in include/woq.h): argument checks, the device
+// check and dispatch to the kernel launchers. Nothing here allocates device memory or
+// synchronises a stream (woq_device_status excepted, which exists to synchronise).
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "woq.h"
+#include "woq_internal.h"
+
+namespace woq {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+DevInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+int g_dev_rc[kMaxDevices];
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_weight(const woq_weight *w) {
+  if (!w || !w->packed || !w->scales) return WOQ_EINVAL;
+  if (w->bits != 4 && w->bits != 8) return WOQ_EINVAL;
+  if (w->block != 32) return WOQ_EINVAL;
+  if (w->n <= 0 || w->k <= 0 || w->k % 32 != 0) return WOQ_ESHAPE;
+  if (w->n > INT32_MAX || w->k > INT32_MAX / 8) return WOQ_ESHAPE;
+  if (!aligned(w->packed, 64) || !aligned(w->scales, 64)) return WOQ_EALIGN;
+  return WOQ_OK;
+}
+
+}  // namespace
+
+void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int current_device(DevInfo *out) {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) return WOQ_ECUDA;
+  if (d < 0 || d >= kMaxDevices) return WOQ_EDEVICE;
+  std::call_once(g_dev_once[d], [d] {
+    DevInfo info;
+    info.device = d;
+    int v = 0;
+    int rc = WOQ_OK;
+    if (cudaDeviceGetAttribute(&info.cc_major, cudaDevAttrComputeCapabilityMajor, d) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.cc_minor, cudaDevAttrComputeCapabilityMinor, d) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, d) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess) {
+      rc = WOQ_ECUDA;
+    } else {
+      info.smem_optin = static_cast<size_t>(v);
+      if (info.cc_major != 10 || info.cc_minor != 0) rc = WOQ_EDEVICE;
+    }
+    g_dev[d] = info;
+    g_dev_rc[d] = rc;
+  });
+  *out = g_dev[d];
+  return g_dev_rc[d];
+}
+
+}  // namespace woq
+
+using woq::DevInfo;
+
+extern "C" {
+
+int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream) {
+  int rc = woq::check_weight(w);
+  if (rc != WOQ_OK) return rc;
+  if (!x || !y) return WOQ_EINVAL;
+  if (m < 1 || m > 64) return WOQ_EINVAL;
+  if (w->k > 32768) return WOQ_ESHAPE;
+  if (!woq::aligned(x, 16) || !woq::aligned(y, 16)) return WOQ_EALIGN;
+  DevInfo dev;
+  rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  return woq::launch_gemv_fp32(x, m, *w, y, static_cast<cudaStream_t>(stream), dev, true);
+}
+
+static int resolve_path(int32_t path, int64_t m) {
+  if (path == WOQ_PATH_AUTO) return m >= 128 ? WOQ_PATH_BF16_TC : WOQ_PATH_FP32;
+  return path;
+}
+
+size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path) {
+  if (woq::check_weight(w) != WOQ_OK || m < 1) return 0;
+  if (path != WOQ_PATH_AUTO && path != WOQ_PATH_FP32 && path != WOQ_PATH_BF16_TC) return 0;
+  return resolve_path(path, m) == WOQ_PATH_BF16_TC ? woq::gemm_tc_workspace_bytes(m, w->k) : 0;
+}
+
+int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path,
+          void *workspace, size_t workspace_bytes, void *stream) {
+  int rc = woq::check_weight(w);
+  if (rc != WOQ_OK) return rc;
+  if (!X || !Y) return WOQ_EINVAL;
+  if (m < 1 || m > INT32_MAX) return WOQ_EINVAL;
+  if (path != WOQ_PATH_AUTO && path != WOQ_PATH_FP32 && path != WOQ_PATH_BF16_TC) return WOQ_EINVAL;
+  if (!woq::aligned(X, 16) || !woq::aligned(Y, 16)) return WOQ_EALIGN;
+  const int p = resolve_path(path, m);
+  if (p == WOQ_PATH_FP32 && w->k > 32768) return WOQ_ESHAPE;
+  if (p == WOQ_PATH_BF16_TC) {
+    const size_t need = woq::gemm_tc_workspace_bytes(m, w->k);
+    if (!workspace || workspace_bytes < need) return WOQ_EWORKSPACE;
+    if (!woq::aligned(workspace, 256)) return WOQ_EALIGN;
+  }
+  DevInfo dev;
+  rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p == WOQ_PATH_FP32) return woq::launch_gemv_fp32(X, m, *w, Y, s, dev, true);
+  return woq::launch_gemm_tc(X, m, *w, Y, workspace, s, dev);
+}
+
+int woq_device_status(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return WOQ_ECUDA;
+  unsigned v = 0;
+  const int rc = woq::read_wait_timeout_flag(clear, &v);
+  if (rc != WOQ_OK) return rc;
+  return v ? WOQ_ETIMEOUT : WOQ_OK;
+}
+
+void woq_debug_set_wait_limit(long long cycles) { woq::set_wait_limit_cycles(cycles); }
+
+const char *woq_status_str(int status) {
+  switch (status) {
+    case WOQ_OK: return "ok";
+    case WOQ_EINVAL: return "invalid argument";
+    case WOQ_ESHAPE: return "unsupported shape";
+    case WOQ_EALIGN: return "misaligned pointer";
+    case WOQ_ERANGE: return "value out of range (non-finite weight or binary16 scale overflow)";
+    case WOQ_EDEVICE: return "device is not compute capability 10.0 (B200)";
+    case WOQ_ECUDA: return "CUDA runtime error";
+    case WOQ_ETIMEOUT: return "a bounded device-side wait gave up";
+    case WOQ_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+uint64_t woq_launch_count(void) { return woq::g_launches.load(std::memory_order_relaxed); }
+
+int woq_abi_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,407 @@
+// FP32 CUDA-core qgemv: y[m, n] = x[m, k] . W_hat^T with W packed int4/int8 in blocks of 32
+// along k and one binary16 scale per block ("TinyMOSS-Diarize", "How we built it": the
+// decode GEMV multiplies straight out of the packed weights, FP32 activations, no
+// dequantised weight tensor).
+//
+// Design (HBM-bound at small m):
+//   * Each warp owns R consecutive weight rows at a time; lane l reads 16-byte chunks
+//     l, l+32, ... of every row (one int4 block or half an int8 block per chunk) with
+//     128-bit streaming loads, so a warp reads 512 contiguous bytes per row per step.
+//   * x rows are staged once per CTA in shared memory, 16-byte units XOR-swizzled so a
+//     quarter-warp reading 8 different chunks hits 8 different bank groups.
+//   * Codes become exact FP32 values with a single LOP3 per element: the 4-bit field
+//     (offset by 8) is placed in the low mantissa bits of 2^23 and the bias is removed
+//     with one exact packed subtraction (f32x2). int4 fields at nibble position j of a
+//     16-bit half carry a factor 2^(4j) that is removed, exactly, once per block.
+//   * Products accumulate per block in FP32 (f32x2 FMA), the block sum is scaled once by
+//     the binary16 scale, and rows are reduced across the warp with shuffles in a fixed
+//     order (deterministic).
+#include <cuda_fp16.h>
+
+#include <mutex>
+#include <unordered_map>
+
+#include "ptx.cuh"
+#include "woq_internal.h"
+
+namespace woq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// 16-byte unit u of an x row lives at unit swz(u) in shared memory.
+__device__ __forceinline__ int swz(int u) { return u ^ ((u >> 3) & 7); }
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// One 32-bit word of int4 codes (elements e0..e7, e_p in bits 4p..4p+3) -> four exact
+// pairs p[j] = (q_j, q_{4+j}) * 2^(4j).
+__device__ __forceinline__ void unpack_int4_word(uint32_t w, float2 (&p)[4]) {
+  const uint32_t hi = w >> 16;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t mask = 0xFu << (4 * j);
+    const uint32_t magic = 0x4B000000u | (0x8u << (4 * j));  // 2^23, field offset by 8
+    const float bias = 8388608.0f + 8.0f * static_cast<float>(1u << (4 * j));
+    const float lo_f = __uint_as_float((w & mask) ^ magic);
+    const float hi_f = __uint_as_float((hi & mask) ^ magic);
+    p[j] = __fadd2_rn(make_float2(lo_f, hi_f), make_float2(-bias, -bias));
+  }
+}
+
+// One 32-bit word of int8 codes (elements e0..e3 in bytes 0..3) -> (q0, q1), (q2, q3).
+__device__ __forceinline__ void unpack_int8_word(uint32_t w, float2 (&p)[2]) {
+  const uint32_t u = w ^ 0x80808080u;  // offset binary, q + 128
+  const float bias = 8388608.0f + 128.0f;
+  const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540));
+  const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541));
+  const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542));
+  const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543));
+  p[0] = __fadd2_rn(make_float2(f0, f1), make_float2(-bias, -bias));
+  p[1] = __fadd2_rn(make_float2(f2, f3), make_float2(-bias, -bias));
+}
+
+__device__ __forceinline__ float fold_int4(const float2 (&a)[4]) {
+  float2 t = __ffma2_rn(a[1], make_float2(0.0625f, 0.0625f), a[0]);
+  t = __ffma2_rn(a[2], make_float2(0.00390625f, 0.00390625f), t);
+  t = __ffma2_rn(a[3], make_float2(0.000244140625f, 0.000244140625f), t);
+  return t.x + t.y;
+}
+
+// int4: one 16-byte chunk (one block of 32) of R rows against MT x rows.
+template <int MT, int R>
+__device__ __forceinline__ void chunk_int4(const float4 *__restrict__ xs4, int units_row, int c,
+                                           const uint4 (&wv)[R], const float (&sc)[R],
+                                           float (&acc)[R][MT]) {
+  if constexpr (MT <= 2) {
+    float4 xv[MT][8];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) xv[mm][t] = xs4[mm * units_row + swz(8 * c + t)];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 a2[MT][4];
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a2[mm][j] = make_float2(0.f, 0.f);
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 p[4];
+        unpack_int4_word(ws[i], p);
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          const float4 xa = xv[mm][2 * i], xb = xv[mm][2 * i + 1];
+          a2[mm][0] = __ffma2_rn(p[0], make_float2(xa.x, xa.y), a2[mm][0]);
+          a2[mm][1] = __ffma2_rn(p[1], make_float2(xa.z, xa.w), a2[mm][1]);
+          a2[mm][2] = __ffma2_rn(p[2], make_float2(xb.x, xb.y), a2[mm][2]);
+          a2[mm][3] = __ffma2_rn(p[3], make_float2(xb.z, xb.w), a2[mm][3]);
+        }
+      }
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], fold_int4(a2[mm]), acc[r][mm]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 p[4][4];
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) unpack_int4_word(ws[i], p[i]);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float2 a2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 xa = xs4[mm * units_row + swz(8 * c + 2 * i)];
+          const float4 xb = xs4[mm * units_row + swz(8 * c + 2 * i + 1)];
+          a2[0] = __ffma2_rn(p[i][0], make_float2(xa.x, xa.y), a2[0]);
+          a2[1] = __ffma2_rn(p[i][1], make_float2(xa.z, xa.w), a2[1]);
+          a2[2] = __ffma2_rn(p[i][2], make_float2(xb.x, xb.y), a2[2]);
+          a2[3] = __ffma2_rn(p[i][3], make_float2(xb.z, xb.w), a2[3]);
+        }
+        acc[r][mm] = fmaf(sc[r], fold_int4(a2), acc[r][mm]);
+      }
+    }
+  }
+}
+
+// int8: one 16-byte chunk (half a block) of R rows against MT x rows.
+template <int MT, int R>
+__device__ __forceinline__ void chunk_int8(const float4 *__restrict__ xs4, int units_row, int c,
+                                           const uint4 (&wv)[R], const float (&sc)[R],
+                                           float (&acc)[R][MT]) {
+  if constexpr (MT <= 2) {
+    float4 xv[MT][4];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) xv[mm][t] = xs4[mm * units_row + swz(4 * c + t)];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 a2[MT];
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) a2[mm] = make_float2(0.f, 0.f);
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 p[2];
+        unpack_int8_word(ws[i], p);
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          a2[mm] = __ffma2_rn(p[0], make_float2(xv[mm][i].x, xv[mm][i].y), a2[mm]);
+          a2[mm] = __ffma2_rn(p[1], make_float2(xv[mm][i].z, xv[mm][i].w), a2[mm]);
+        }
+      }
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], a2[mm].x + a2[mm].y, acc[r][mm]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 p[4][2];
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) unpack_int8_word(ws[i], p[i]);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 xa = xs4[mm * units_row + swz(4 * c + i)];
+          a2 = __ffma2_rn(p[i][0], make_float2(xa.x, xa.y), a2);
+          a2 = __ffma2_rn(p[i][1], make_float2(xa.z, xa.w), a2);
+        }
+        acc[r][mm] = fmaf(sc[r], a2.x + a2.y, acc[r][mm]);
+      }
+    }
+  }
+}
+
+// grid.x: CTAs striding over units of R rows; grid.y: passes of MT x rows.
+template <int BITS, int MT, int R, int U>
+__global__ void __launch_bounds__(kThreads)
+    gemv_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
+                const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n, int k) {
+  extern __shared__ float4 xs4[];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int m0 = blockIdx.y * MT;
+  const int units_row = k >> 2;
+
+  // Everything below reads x or writes y, which a preceding kernel may produce or read.
+  ptx::pdl_wait();
+
+  // Stage x rows [m0, m0 + MT): 8-element groups; int4 interleaves (0,4,1,5 | 2,6,3,7)
+  // so that each f32x2 pair lines up with the code pair (q_j, q_{4+j}).
+  const int groups = k >> 3;
+  for (int idx = tid; idx < MT * groups; idx += kThreads) {
+    const int mm = idx / groups;
+    const int g = idx - mm * groups;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (m0 + mm < m) {
+      const float4 *src = reinterpret_cast<const float4 *>(x + static_cast<size_t>(m0 + mm) * k) + 2 * g;
+      a = src[0];
+      b = src[1];
+    }
+    float4 pa = a, pb = b;
+    if constexpr (BITS == 4) {
+      pa = make_float4(a.x, b.x, a.y, b.y);
+      pb = make_float4(a.z, b.z, a.w, b.w);
+    }
+    float4 *row = xs4 + mm * units_row;
+    row[swz(2 * g)] = pa;
+    row[swz(2 * g + 1)] = pb;
+  }
+  __syncthreads();
+  ptx::pdl_launch_dependents();
+
+  const int cpr = (k * BITS) >> 7;  // 16-byte chunks per weight row
+  const int spr = k >> 5;           // scales per row
+  const size_t row_bytes = static_cast<size_t>(k) * BITS / 8;
+  const int units = (n + R - 1) / R;
+
+  for (int unit = blockIdx.x * kWarps + warp; unit < units; unit += gridDim.x * kWarps) {
+    const int row0 = unit * R;
+    float acc[R][MT];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = 0.f;
+
+    for (int cb = 0; cb < cpr; cb += 32 * U) {
+      uint4 wv[U][R];
+      float sc[U][R];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = cb + 32 * u + lane;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int row = row0 + r;
+          if (c < cpr && row < n) {
+            wv[u][r] = ptx::ldg_stream_v4(packed + static_cast<size_t>(row) * row_bytes +
+                                          static_cast<size_t>(c) * 16);
+            sc[u][r] = half_bits_to_float(
+                __ldg(scales + static_cast<size_t>(row) * spr + (BITS == 4 ? c : (c >> 1))));
+          } else {
+            wv[u][r] = make_uint4(0u, 0u, 0u, 0u);
+            sc[u][r] = 0.f;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = cb + 32 * u + lane;
+        if (c < cpr) {
+          if constexpr (BITS == 4)
+            chunk_int4<MT, R>(xs4, units_row, c, wv[u], sc[u], acc);
+          else
+            chunk_int8<MT, R>(xs4, units_row, c, wv[u], sc[u], acc);
+        }
+      }
+    }
+
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float v = acc[r][mm];
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        acc[r][mm] = v;
+      }
+    // Lane (r * MT + mm) stores one result.
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm)
+        if (lane == r * MT + mm && row0 + r < n && m0 + mm < m)
+          y[static_cast<size_t>(m0 + mm) * n + row0 + r] = acc[r][mm];
+  }
+}
+
+struct OccKey {
+  const void *fn;
+  size_t smem;
+  int device;
+  bool operator==(const OccKey &o) const {
+    return fn == o.fn && smem == o.smem && device == o.device;
+  }
+};
+struct OccHash {
+  size_t operator()(const OccKey &k) const {
+    return std::hash<const void *>()(k.fn) ^ (k.smem * 1315423911u) ^ (size_t(k.device) << 48);
+  }
+};
+
+// Resident CTAs per SM for (kernel, dynamic smem) on the device; also raises the
+// kernel's dynamic shared memory limit when needed. Cached.
+int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev) {
+  static std::mutex mu;
+  static std::unordered_map<OccKey, int, OccHash> cache;
+  const OccKey key{fn, smem, dev.device};
+  {
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -1;
+  }
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, smem) != cudaSuccess)
+    return -1;
+  std::lock_guard<std::mutex> g(mu);
+  cache[key] = nb;
+  return nb;
+}
+
+template <int BITS, int MT, int R, int U>
+int launch_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+             const DevInfo &dev, bool pdl) {
+  auto kern = gemv_kernel<BITS, MT, R, U>;
+  const size_t smem = static_cast<size_t>(MT) * w.k * sizeof(float);
+  const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev);
+  if (nb <= 0) return WOQ_ECUDA;
+  const int64_t units = (w.n + R - 1) / R;
+  int64_t gx = (units + kWarps - 1) / kWarps;
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * nb;
+  if (gx > cap) gx = cap;
+  const int64_t gy = (m + MT - 1) / MT;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, w.packed, w.scales, y, static_cast<int>(m),
+                                           static_cast<int>(w.n), static_cast<int>(w.k));
+  if (e != cudaSuccess) return WOQ_ECUDA;
+  count_launches(1);
+  return WOQ_OK;
+}
+
+template <int BITS, int MT>
+int pick_ru(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+            const DevInfo &dev, bool pdl) {
+  const int64_t cpr = w.k * BITS / 128;
+  const bool two = cpr > 32;
+  // Enough warps to cover the machine a few times over with R rows each.
+  const int64_t want = static_cast<int64_t>(dev.sm_count) * 16;
+  int R = 1;
+  if (MT <= 2) {
+    if ((w.n + 3) / 4 >= want) R = 4;
+    else if ((w.n + 1) / 2 >= want) R = 2;
+  } else if ((w.n + 1) / 2 >= want) {
+    R = 2;
+  }
+  if constexpr (MT <= 2) {
+    if (R == 4) return two ? launch_t<BITS, MT, 4, 2>(x, m, w, y, s, dev, pdl)
+                           : launch_t<BITS, MT, 4, 1>(x, m, w, y, s, dev, pdl);
+  }
+  if (R == 2) return two ? launch_t<BITS, MT, 2, 2>(x, m, w, y, s, dev, pdl)
+                         : launch_t<BITS, MT, 2, 1>(x, m, w, y, s, dev, pdl);
+  return two ? launch_t<BITS, MT, 1, 2>(x, m, w, y, s, dev, pdl)
+             : launch_t<BITS, MT, 1, 1>(x, m, w, y, s, dev, pdl);
+}
+
+template <int BITS>
+int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+            const DevInfo &dev, bool pdl) {
+  int mt = m == 1 ? 1 : m == 2 ? 2 : m <= 4 ? 4 : 8;
+  const size_t limit = dev.smem_optin < 200 * 1024 ? dev.smem_optin : 200 * 1024;
+  while (mt > 1 && static_cast<size_t>(mt) * w.k * sizeof(float) > limit) mt /= 2;
+  if (static_cast<size_t>(mt) * w.k * sizeof(float) > limit) return WOQ_ESHAPE;
+  switch (mt) {
+    case 1: return pick_ru<BITS, 1>(x, m, w, y, s, dev, pdl);
+    case 2: return pick_ru<BITS, 2>(x, m, w, y, s, dev, pdl);
+    case 4: return pick_ru<BITS, 4>(x, m, w, y, s, dev, pdl);
+    default: return pick_ru<BITS, 8>(x, m, w, y, s, dev, pdl);
+  }
+}
+
+}  // namespace
+
+int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                     const DevInfo &dev, bool pdl) {
+  return w.bits == 4 ? pick_mt<4>(x, m, w, y, s, dev, pdl) : pick_mt<8>(x, m, w, y, s, dev, pdl);
+}
+
+}  // namespace woq

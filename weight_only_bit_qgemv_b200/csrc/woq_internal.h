@@ -1,0 +1,45 @@
+// Internal interfaces between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "woq.h"
+
+namespace woq {
+
+struct DevInfo {
+  int device = -1;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  size_t smem_optin = 0;  // max dynamic shared memory per block (opt-in)
+};
+
+// Properties of the current device (cached per device). WOQ_EDEVICE unless it is
+// compute capability 10.0; WOQ_ECUDA if the runtime cannot be queried.
+int current_device(DevInfo *out);
+
+// Adds n to the process-wide launch counter reported by woq_launch_count().
+void count_launches(uint64_t n);
+
+// ---- qgemv.cu ----
+// FP32 CUDA-core GEMV/GEMM: y[m, n] = x[m, k] . W_hat^T for any m >= 1. Arguments
+// already validated. `pdl` launches with programmatic stream serialization.
+int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                     const DevInfo &dev, bool pdl);
+
+// ---- qgemm_tc.cu ----
+// Workspace bytes of the tensor-core path (the bf16 copy of X).
+size_t gemm_tc_workspace_bytes(int64_t m, int64_t k);
+// tcgen05 bf16 GEMM: Y = bf16(X) . bf16(W_hat)^T, FP32 accumulation in tensor memory.
+int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
+                   cudaStream_t s, const DevInfo &dev);
+// Reads (and optionally clears) the device-side record of bounded waits that gave up on
+// the current device. Synchronous.
+int read_wait_timeout_flag(int clear, unsigned *value);
+// Test hook: cycle budget of every bounded wait in the tensor-core kernel (0 = default).
+void set_wait_limit_cycles(long long cycles);
+
+}  // namespace woq
