@@ -145,11 +145,14 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
 int woq_device_status(int clear);
 
 /*
- * woq_debug_set_wait_limit -- test hook. Sets the cycle budget of every bounded wait in the
- * tensor-core qgemm kernel for launches that follow: cycles > 0 sets it, cycles < 0 makes
- * every wait that would have to spin give up at once (so the timeout path can be exercised
- * without a hang), 0 restores the default (2^32 cycles, about two seconds). Host-side state
- * of the process, not thread-safe against concurrent launches.
+ * woq_debug_set_wait_limit -- test hook for the tensor-core qgemm kernel's bounded waits,
+ * applied to launches that follow. cycles > 0 sets the cycle budget of every wait;
+ * 0 restores the default (2^32 cycles, about two seconds); cycles < 0 keeps the default
+ * and makes the MMA-issuing thread of every CTA first wait on a barrier that nothing
+ * arrives on, bounded by -cycles cycles, so the give-up path runs deterministically
+ * without a hang (the kernel then records the event, drains, frees tensor memory and
+ * returns; woq_device_status reports WOQ_ETIMEOUT). Process-wide host state; not
+ * thread-safe against concurrent launches.
  */
 void woq_debug_set_wait_limit(long long cycles);
 

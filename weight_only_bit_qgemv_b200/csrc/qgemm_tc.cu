@@ -37,7 +37,7 @@ constexpr int kThreads = 64 + kDequantWarps * 32;  // 320
 constexpr long long kDrainLimit = 1LL << 31;       // cycles (~1 s) for draining on abort
 constexpr long long kDefaultWaitLimit = 1LL << 32;  // cycles (~2 s) for ordinary waits
 
-long long g_wait_limit_cycles = 0;  // test hook; 0 = default
+long long g_wait_limit_cycles = 0;  // test hook: > 0 wait limit, < 0 inject a stuck wait
 
 template <int BITS, int BN>
 struct Cfg {
@@ -69,6 +69,7 @@ struct Shared {
   uint64_t bfull[kStages];  // bf16 weight tile written by the dequantisers
   uint64_t empty[kStages];  // MMAs reading the stage completed
   uint64_t acc_full;        // all MMAs of the tile completed
+  uint64_t never;           // nothing arrives here: target of the injected stuck wait
   uint32_t tmem_base;
   int abort;
 };
@@ -132,7 +133,7 @@ template <int BITS, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const uint16_t *__restrict__ scales, float *__restrict__ Y, int M, int N, int K,
-                    long long wait_limit) {
+                    long long wait_limit, long long stuck_wait) {
   using C = Cfg<BITS, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&sh.empty[s], 1);
     }
     ptx::mbar_init(&sh.acc_full, 1);
+    ptx::mbar_init(&sh.never, 1);
     sh.abort = 0;
     ptx::fence_mbar_init();
   }
@@ -194,6 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = true;
+      // Test hook: a wait on a barrier nothing arrives on, which must run out.
+      if (stuck_wait > 0 && !ptx::mbar_wait_bounded(&sh.never, 0, stuck_wait, abort)) {
+        record_timeout(abort);
+        ok = false;
+      }
       for (int ks = 0; ks < num_k && ok; ++ks) {
         const int s = ks % kStages;
         const uint32_t ph = (ks / kStages) & 1;
@@ -437,11 +444,10 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const long long lim = g_wait_limit_cycles > 0 ? g_wait_limit_cycles
-                          : g_wait_limit_cycles < 0 ? 0
-                                                    : kDefaultWaitLimit;
+    const long long lim = g_wait_limit_cycles > 0 ? g_wait_limit_cycles : kDefaultWaitLimit;
+    const long long stuck = g_wait_limit_cycles < 0 ? -g_wait_limit_cycles : 0;
     if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, w.scales, Y, static_cast<int>(m),
-                           static_cast<int>(w.n), static_cast<int>(w.k), lim) != cudaSuccess)
+                           static_cast<int>(w.n), static_cast<int>(w.k), lim, stuck) != cudaSuccess)
       return WOQ_ECUDA;
     count_launches(1);
   }
