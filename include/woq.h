@@ -137,6 +137,30 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * qgemm_bf16_noalloc -- the WOQ_PATH_BF16_TC qgemm for callers that cannot allocate device
+ * memory. The pages have no counterpart to this call; it exists for integration.
+ * Who needs it: a caller that can pass its input and output buffers but has no way to
+ * obtain a workspace -- a plugin whose host hands it only its tensors, a serving runtime
+ * that has reserved all device memory for its own pool and forbids other allocations, or
+ * a latency-critical loop that cannot afford cudaMalloc's implicit device-wide
+ * synchronisation.
+ * Instead of a caller workspace it uses one fixed 32 MiB scratch array compiled into the
+ * library (a __device__ symbol; every GPU that loads the library holds it until the
+ * process exits). It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * call. Arguments, result and arithmetic are those of qgemm with path WOQ_PATH_BF16_TC.
+ *   X, m, w, Y, stream  as for qgemm
+ * Limit: m * k * 2 bytes (the bf16 copy of X, rounded up to 256) must not exceed 32 MiB,
+ *   e.g. m <= 4096 at k = 4096; larger problems return WOQ_ESHAPE and queue nothing.
+ * The first call on each device looks up the scratch array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * All calls on a device share the scratch array. Each call overwrites the part it reads
+ * before reading it, so nothing needs clearing, but two calls whose kernels overlap on the
+ * GPU (e.g. on unordered streams) race on it: order them on one stream.
+ * Errors: those of qgemm, with WOQ_ESHAPE also for the size limit.
+ */
+int qgemm_bf16_noalloc(const float *X, int64_t m, const woq_weight *w, float *Y, void *stream);
+
+/*
  * woq_device_status -- synchronises the current device, then returns WOQ_ETIMEOUT if any
  * kernel of this library recorded a bounded wait that gave up since the last call with
  * clear != 0 (and clears the record if clear != 0), WOQ_ECUDA if synchronisation failed,

@@ -28,6 +28,7 @@ EXPORTS = (
     "qgemv",
     "qgemm_workspace_bytes",
     "qgemm",
+    "qgemm_bf16_noalloc",
     "woq_device_status",
     "woq_debug_set_wait_limit",
     "woq_status_str",
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.qgemm_workspace_bytes.restype = ctypes.c_size_t
     L.qgemm.argtypes = [vp, c_i64, wp, vp, c_i32, vp, ctypes.c_size_t, vp]
     L.qgemm.restype = ctypes.c_int
+    L.qgemm_bf16_noalloc.argtypes = [vp, c_i64, wp, vp, vp]
+    L.qgemm_bf16_noalloc.restype = ctypes.c_int
     L.woq_device_status.argtypes = [ctypes.c_int]
     L.woq_device_status.restype = ctypes.c_int
     L.woq_debug_set_wait_limit.argtypes = [ctypes.c_longlong]

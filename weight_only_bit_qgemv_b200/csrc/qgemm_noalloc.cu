@@ -1,0 +1,72 @@
+// qgemm_bf16_noalloc: the tensor-core qgemm for callers that cannot allocate device memory.
+//
+// The ordinary qgemm asks its caller for a workspace (the bf16 copy of X that the tensor
+// cores read). Some callers have no way to provide one: a plugin whose host hands it only
+// its input and output buffers, a serving runtime that has already reserved all device
+// memory for its own pool and forbids any other allocation, or a latency-critical loop in
+// which cudaMalloc's implicit device-wide synchronisation cannot be afforded. For them this
+// entry point uses a fixed scratch array that lives in the library's own device image.
+//
+// That array is a file-scope __device__ symbol of kScratchBytes (32 MiB). Every GPU that
+// loads the library holds it until the process exits. In host code its name is only a
+// host-side stand-in for the symbol, never a device address, so the real address is
+// looked up once per device with cudaGetSymbolAddress (with that device current) and
+// cached. All calls on a device share the one array; its contents after a call are that
+// call's bf16 copy of X, and every call overwrites the part it reads before reading it, so
+// nothing has to be cleared. Two calls whose kernels overlap on the GPU (for example on two
+// streams without ordering between them) race on the array.
+#include <mutex>
+
+#include "woq.h"
+#include "woq_internal.h"
+
+namespace woq {
+namespace {
+
+constexpr size_t kScratchBytes = size_t(32) << 20;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+void *g_ptr[kMaxDevices];
+int g_rc[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up once per device).
+int scratch_address(int device, void **out) {
+  if (device < 0 || device >= kMaxDevices) return WOQ_EDEVICE;
+  std::call_once(g_once[device], [device] {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_ptr[device] = p;
+    g_rc[device] = (e == cudaSuccess && p != nullptr) ? WOQ_OK : WOQ_ECUDA;
+  });
+  *out = g_ptr[device];
+  return g_rc[device];
+}
+
+}  // namespace
+}  // namespace woq
+
+extern "C" int qgemm_bf16_noalloc(const float *X, int64_t m, const woq_weight *w, float *Y,
+                                  void *stream) {
+  if (!w || !w->packed || !w->scales) return WOQ_EINVAL;
+  if (w->bits != 4 && w->bits != 8) return WOQ_EINVAL;
+  if (w->block != 32) return WOQ_EINVAL;
+  if (w->n <= 0 || w->k <= 0 || w->k % 32 != 0) return WOQ_ESHAPE;
+  if (w->n > INT32_MAX || w->k > INT32_MAX / 8) return WOQ_ESHAPE;
+  if (!X || !Y) return WOQ_EINVAL;
+  if (m < 1 || m > INT32_MAX) return WOQ_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(w->packed) & 63) || (reinterpret_cast<uintptr_t>(w->scales) & 63))
+    return WOQ_EALIGN;
+  if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(Y) & 15)) return WOQ_EALIGN;
+  // The bf16 copy of X must fit in the fixed scratch array.
+  if (woq::gemm_tc_workspace_bytes(m, w->k) > woq::kScratchBytes) return WOQ_ESHAPE;
+  woq::DevInfo dev;
+  int rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  void *scratch = nullptr;
+  rc = woq::scratch_address(dev.device, &scratch);
+  if (rc != WOQ_OK) return rc;
+  return woq::launch_gemm_tc(X, m, *w, Y, scratch, static_cast<cudaStream_t>(stream), dev);
+}
