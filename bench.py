@@ -4,10 +4,12 @@
 
 Default workload ("decoder_block_m1"): one Qwen3-0.6B-style decoder block at decode, M = 1,
 int4 block-32 weights: the 7 projections q[2048x1024], k[1024x1024], v[1024x1024],
-o[1024x2048], gate/up[3072x1024], down[1024x3072]. One step runs the 7 qgemv calls of one
-block; consecutive steps walk the 28 blocks of a seeded synthetic decoder (247.7 MB of
-packed weights, more than the 126 MB L2), so every step streams its weights from HBM.
-Metric: weight GB/s (packed codes + scales per step / time).
+o[1024x2048], gate/up[3072x1024], down[1024x3072]. q|k|v share their input, as do gate|up,
+so their packed rows are stored concatenated and one step is 4 qgemv calls: qkv[4096x1024],
+o, gate_up[6144x1024], down (--unfused: 7 calls). Consecutive steps walk the 28 blocks of a
+seeded synthetic decoder (247.7 MB of packed weights, more than the 126 MB L2), so every
+step streams its weights from HBM. Metric: weight GB/s (packed codes + scales per step /
+time).
 
 Timed region: K steps replayed from CUDA graphs on one stream, bracketed by a barrier and
 device synchronisation, timed with CUDA events on that stream; the max over ranks is
@@ -16,8 +18,10 @@ reported. Under torchrun every rank runs its own replica (no data-path collectiv
 Also on the JSON line: `e2e` (the same steps through the public API with x copied from
 pinned host memory and y read back every step), `roofline` (the qgemv kernel against the
 measured HBM copy bandwidth), `cpu_baseline` (the CPU oracle on the host cores, a bounded
-sample), `parity` (GPU vs oracle on the sampled step), and `prefill` (the tcgen05 qgemm over
-all 7 projections of all 28 blocks at M = 512, TFLOP/s against the measured bf16 peak).
+sample), `parity` (GPU vs oracle on the sampled step), `kernel_roofline_lm_head` (one qgemv
+launch over the 165 MB int8 lm_head, the kernel alone against HBM), and `prefill` (the tcgen05
+qgemm over all projections of all 28 blocks at M = 512, TFLOP/s against the measured bf16
+peak).
 """
 
 from __future__ import annotations
@@ -164,17 +168,38 @@ class ClockSampler:
 # the workload
 # --------------------------------------------------------------------------------------
 
-def build_decoder(bits: int, device, n_layers: int = workloads.N_LAYERS):
+#: Launch groups of one decoder block. A real decoder feeds q, k and v the same input and
+#: gate and up the same input, so their weights are stored row-concatenated and run as one
+#: qgemv each (qkv [4096x1024], gate_up [6144x1024]); every packed byte is unchanged.
+FUSED_GROUPS = (("qkv", (0, 1, 2)), ("o", (3,)), ("gate_up", (4, 5)), ("down", (6,)))
+UNFUSED_GROUPS = tuple((nm, (i,)) for i, (nm, _, _) in enumerate(workloads.DECODER_PROJ))
+
+
+def group_shape(members):
+    n = sum(workloads.DECODER_PROJ[i][1] for i in members)
+    k = workloads.DECODER_PROJ[members[0]][2]
+    return n, k
+
+
+def group_x_seed(members):
+    """Activation seed of a launch group (one input per group, shared by its members)."""
+    return workloads.X_SEED + members[0]
+
+
+def group_weight(layer, members):
+    """float32 weight of a group: its members' seeded weights, rows concatenated."""
+    ws = []
+    for i in members:
+        _, n, k = workloads.DECODER_PROJ[i]
+        ws.append(workloads.weight(n, k, seed=workloads.layer_seed(layer, i)))
+    return torch.cat(ws, 0) if len(ws) > 1 else ws[0]
+
+
+def build_decoder(bits: int, device, groups, n_layers: int = workloads.N_LAYERS):
     import weight_only_bit_qgemv_b200 as woq
 
-    layers = []
-    for layer in range(n_layers):
-        projs = []
-        for p, (_, n, k) in enumerate(workloads.DECODER_PROJ):
-            W = workloads.weight(n, k, seed=workloads.layer_seed(layer, p))
-            projs.append(woq.pack(W, bits, device))
-        layers.append(projs)
-    return layers
+    return [[woq.pack(group_weight(layer, mem), bits, device) for _, mem in groups]
+            for layer in range(n_layers)]
 
 
 def decode_step_bytes(layer):
@@ -237,16 +262,17 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
 
     device = torch.device("cuda", local)
     bits = 4
-    layers = build_decoder(bits, device)
-    xs = [workloads.activations(1, k, seed=workloads.X_SEED + p).to(device)
-          for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
-    ys = [torch.empty(1, n, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    groups = UNFUSED_GROUPS if args.unfused else FUSED_GROUPS
+    layers = build_decoder(bits, device, groups)
+    xs = [workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
+          for _, mem in groups]
+    ys = [torch.empty(1, group_shape(mem)[0], device=device) for _, mem in groups]
     step_bytes = decode_step_bytes(layers[0])
     total_bytes = sum(decode_step_bytes(l) for l in layers)
 
     def step(i):
-        for p, w in enumerate(layers[i]):
-            woq.qgemv(xs[p], w, out=ys[p])
+        for g, w in enumerate(layers[i]):
+            woq.qgemv(xs[g], w, out=ys[g])
 
     stream = torch.cuda.Stream(device)
     with ClockSampler(local) as clk:
@@ -264,7 +290,7 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
                 "bytes_per_launch": round(step_bytes / per_step),
                 "avg_launch_us": round(ms * 1e3 / launches, 3)}
 
-    e2e = run_decode_e2e(layers, device, min(args.steps, 2000), stream, world)
+    e2e = run_decode_e2e(layers, groups, device, min(args.steps, 2000), stream, world)
 
     out = {
         "metric": "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)",
@@ -272,7 +298,9 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "decoder_block_m1", "bits": 4, "block": 32, "m": 1,
-                   "projections": [f"{nm}[{n}x{k}]" for nm, n, k in workloads.DECODER_PROJ],
+                   "launches": [f"{nm}[{group_shape(mem)[0]}x{group_shape(mem)[1]}]"
+                                for nm, mem in groups],
+                   "fused_qkv_gate_up": not args.unfused,
                    "layers_cycled": len(layers), "weight_bytes_per_step": step_bytes,
                    "l2": f"inputs larger than L2: steps walk {len(layers)} blocks, "
                          f"{total_bytes / 1e6:.1f} MB of packed weights > 126 MB L2",
@@ -284,26 +312,26 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
         "gpu_launches": int(launches),
         "roofline": roofline,
     }
-    return out, layers, xs, ys
+    return out, layers, groups, xs
 
 
-def run_decode_e2e(layers, device, steps, stream, world):
+def run_decode_e2e(layers, groups, device, steps, stream, world):
     """Same steps through the public API, x from pinned host memory, y read back each step."""
     import weight_only_bit_qgemv_b200 as woq
 
-    host_x = [workloads.activations(1, k, seed=workloads.X_SEED + p).pin_memory()
-              for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
-    host_y = [torch.empty(1, n).pin_memory() for (_, n, k) in workloads.DECODER_PROJ]
-    dx = [torch.empty(1, k, device=device) for (_, n, k) in workloads.DECODER_PROJ]
-    dy = [torch.empty(1, n, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    host_x = [workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).pin_memory()
+              for _, mem in groups]
+    host_y = [torch.empty(1, group_shape(mem)[0]).pin_memory() for _, mem in groups]
+    dx = [torch.empty_like(h, device=device) for h in host_x]
+    dy = [torch.empty_like(h, device=device) for h in host_y]
     h2d = sum(t.numel() * 4 for t in host_x)
     d2h = sum(t.numel() * 4 for t in host_y)
 
     def step(i):
-        for p, w in enumerate(layers[i % len(layers)]):
-            dx[p].copy_(host_x[p], non_blocking=True)
-            woq.qgemv(dx[p], w, out=dy[p])
-            host_y[p].copy_(dy[p], non_blocking=True)
+        for g, w in enumerate(layers[i % len(layers)]):
+            dx[g].copy_(host_x[g], non_blocking=True)
+            woq.qgemv(dx[g], w, out=dy[g])
+            host_y[g].copy_(dy[g], non_blocking=True)
         stream.synchronize()
 
     with torch.cuda.stream(stream):
@@ -325,26 +353,58 @@ def run_decode_e2e(layers, device, steps, stream, world):
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps}
 
 
-def run_prefill(layers, device, m: int, reps: int, peaks, peak_kind, world):
-    """tcgen05 qgemm through all 7 projections of all blocks at M = m (one pass = one rep)."""
+def run_lm_head_roofline(device, peaks, peak_kind, reps=20):
+    """qgemv on the int8 lm_head [151936x1024] at M = 1: one 165 MB launch, the kernel alone.
+
+    Two packed copies alternate so that every launch streams its weights from HBM.
+    """
     import weight_only_bit_qgemv_b200 as woq
 
-    Xs = [workloads.activations(m, k, seed=workloads.X_SEED + p).to(device)
-          for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
-    Ys = [torch.empty(m, n, device=device) for (_, n, k) in workloads.DECODER_PROJ]
+    n, k = workloads.LM_HEAD
+    w0 = woq.pack(workloads.weight(n, k, seed=workloads.LM_HEAD_SEED), 8, device)
+    w1 = woq.PackedWeight(w0.packed.clone(), w0.scales.clone(), 8, n, k)
+    x = workloads.activations(1, k, seed=workloads.X_SEED).to(device)
+    y = torch.empty(1, n, device=device)
+    for _ in range(3):
+        woq.qgemv(x, w0, out=y)
+        woq.qgemv(x, w1, out=y)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    s = torch.cuda.current_stream()
+    ev[0].record(s)
+    for r in range(reps):
+        woq.qgemv(x, w0 if r % 2 == 0 else w1, out=y)
+        ev[r + 1].record(s)
+    ev[-1].synchronize()
+    times = [ev[r].elapsed_time(ev[r + 1]) for r in range(reps)]
+    med = statistics.median(times)
+    gbs = w0.nbytes / (med / 1e3) / 1e9
+    return {"workload": "lm_head_m1_int8", "weight_bytes": w0.nbytes, "launch_us_median": med * 1e3,
+            "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peak_kind,
+            "timing": f"median of {reps} single launches, CUDA events, two alternating copies"}
+
+
+def run_prefill(layers, groups, device, m: int, reps: int, peaks, peak_kind, world):
+    """tcgen05 qgemm through every projection of every block at M = m (one pass = one rep)."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    Xs = [workloads.activations(m, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
+          for _, mem in groups]
+    Ys = [torch.empty(m, group_shape(mem)[0], device=device) for _, mem in groups]
     ws = torch.empty(max(woq.qgemm_workspace_bytes(m, w, "bf16_tc") for w in layers[0]),
                      dtype=torch.uint8, device=device)
     flops = 2.0 * m * sum(n * k for _, n, k in workloads.DECODER_PROJ) * len(layers)
 
     def step(i):
         for layer in layers:
-            for p, w in enumerate(layer):
-                woq.qgemm(Xs[p], w, path="bf16_tc", out=Ys[p], workspace=ws)
+            for g, w in enumerate(layer):
+                woq.qgemm(Xs[g], w, path="bf16_tc", out=Ys[g], workspace=ws)
 
     stream = torch.cuda.Stream(device)
     ms, per_step = time_graph_steps(step, 1, reps, 2, stream, world)
     tflops = flops * reps / (ms / 1e3) / 1e12
-    return {"workload": f"prefill_m{m}", "m": m, "gemms_per_pass": len(layers) * 7,
+    return {"workload": f"prefill_m{m}", "m": m, "gemm_calls_per_pass": len(layers) * len(groups),
             "flop_per_pass": flops, "passes": reps, "ms_per_pass": ms / reps,
             "tflops": round(tflops, 1), "peak_tflops": peaks["bf16_tflops"],
             "frac": round(tflops / peaks["bf16_tflops"], 4), "peak_source": peak_kind,
@@ -367,18 +427,22 @@ def oracle_decode_pass(packed_layer, xs_np, rows=None):
     return outs
 
 
-def oracle_layer_inputs(bits=4, layer=0):
-    """Packed weights of one block, quantised and packed by the oracle itself, and x rows."""
+def oracle_layer_inputs(groups, bits=4, layer=0):
+    """The block's 7 projections, quantised and packed by the oracle itself, and their x rows
+    (members of a launch group share its input)."""
     import oracle
 
+    x_of = {}
+    for _, mem in groups:
+        x = workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).numpy()
+        for i in mem:
+            x_of[i] = x
     out = []
     for p, (_, n, k) in enumerate(workloads.DECODER_PROJ):
         W = workloads.weight(n, k, seed=workloads.layer_seed(layer, p)).numpy()
         q, s = oracle.quantise(W, bits)
         out.append((oracle.pack(q, bits), s, bits))
-    xs = [workloads.activations(1, k, seed=workloads.X_SEED + p).numpy()
-          for p, (_, n, k) in enumerate(workloads.DECODER_PROJ)]
-    return out, xs
+    return out, [x_of[p] for p in range(len(workloads.DECODER_PROJ))]
 
 
 def blas_threads():
@@ -405,23 +469,23 @@ def time_oracle(packed_layer, xs, budget_s: float):
     return statistics.median(times), len(times), outs
 
 
-def cpu_baseline_leg(layer0_gpu, xs_gpu, budget_s):
+def cpu_baseline_leg(layer0_gpu, groups, xs_gpu, budget_s):
     import weight_only_bit_qgemv_b200 as woq
 
-    packed, xs = oracle_layer_inputs()
+    packed, xs = oracle_layer_inputs(groups)
     sec, passes, outs = time_oracle(packed, xs, budget_s)
     nbytes = sum(pk.nbytes + sc.nbytes for pk, sc, _ in packed)
     # parity of the GPU step against the oracle on the same inputs (block 0)
     errs = []
-    for p, w in enumerate(layer0_gpu):
-        y = woq.qgemv(xs_gpu[p], w).cpu().numpy()
-        ref = outs[p]
+    for g, (w, (_, mem)) in enumerate(zip(layer0_gpu, groups)):
+        y = woq.qgemv(xs_gpu[g], w).cpu().numpy()
+        ref = np.concatenate([outs[i] for i in mem], axis=1)
         errs.append(float(np.max(np.abs(y - ref)) / np.max(np.abs(ref))))
     return ({"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
              "kind": "oracle",
              "sample": f"{passes} passes of decoder block 0 (7 projections, M=1, int4) through the "
                        f"NumPy float64 oracle, median pass {sec * 1e3:.1f} ms"},
-            {"max_rel_err": max(errs), "tolerance": 1e-4, "checked": "block 0, all 7 outputs"})
+            {"max_rel_err": max(errs), "tolerance": 1e-4, "checked": "block 0, every output"})
 
 
 def run_reference(args, world, rank, budget_s=90.0):
@@ -433,7 +497,7 @@ def run_reference(args, world, rank, budget_s=90.0):
     """
     if rank != 0:
         return None
-    packed, xs = oracle_layer_inputs()
+    packed, xs = oracle_layer_inputs(FUSED_GROUPS)
     t0 = time.perf_counter()
     oracle_decode_pass(packed, xs)
     full = time.perf_counter() - t0
@@ -475,6 +539,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-m", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--unfused", action="store_true", help="7 launches per block instead of 4")
+    ap.add_argument("--no-lm-head", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -490,12 +556,15 @@ def main(argv=None):
         print(json.dumps({"error": "no CUDA device"}))
         return 1
     peaks, peak_kind = load_peaks()
-    out, layers, xs, ys = run_decode(args, world, rank, local, peaks, peak_kind)
+    out, layers, groups, xs = run_decode(args, world, rank, local, peaks, peak_kind)
+    device = torch.device("cuda", local)
+    if not args.no_lm_head:
+        out["kernel_roofline_lm_head"] = run_lm_head_roofline(device, peaks, peak_kind)
     if not args.no_prefill:
-        out["prefill"] = run_prefill(layers, torch.device("cuda", local), args.prefill_m, 3,
-                                     peaks, peak_kind, world)
-    if rank == 0 and world >= 1 and not args.no_cpu_baseline:
-        cb, parity = cpu_baseline_leg(layers[0], xs, args.cpu_budget)
+        out["prefill"] = run_prefill(layers, groups, device, args.prefill_m, 3, peaks, peak_kind,
+                                     world)
+    if rank == 0 and not args.no_cpu_baseline:
+        cb, parity = cpu_baseline_leg(layers[0], groups, xs, args.cpu_budget)
         out["cpu_baseline"] = cb
         out["parity"] = parity
     if rank == 0:

@@ -114,10 +114,12 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
 
 int woq_device_status(int clear) {
   if (cudaDeviceSynchronize() != cudaSuccess) return WOQ_ECUDA;
-  unsigned v = 0;
-  const int rc = woq::read_wait_timeout_flag(clear, &v);
+  unsigned v = 0, g = 0;
+  int rc = woq::read_wait_timeout_flag(clear, &v);
   if (rc != WOQ_OK) return rc;
-  return v ? WOQ_ETIMEOUT : WOQ_OK;
+  rc = woq::read_gemv_timeout_flag(clear, &g);
+  if (rc != WOQ_OK) return rc;
+  return (v || g) ? WOQ_ETIMEOUT : WOQ_OK;
 }
 
 void woq_debug_set_wait_limit(long long cycles) { woq::set_wait_limit_cycles(cycles); }

@@ -18,6 +18,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "ptx.cuh"
@@ -32,6 +33,8 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;           // bf16 elements per stage = one 128-byte swizzle row
 constexpr int kStages = 4;
+constexpr int kWinStages = 32;   // K-stages whose scales each dequantiser holds in shared memory
+constexpr int kTmaScaleCols = 128;  // scale tile copied whole by TMA when K/32 <= this
 constexpr int kDequantWarps = 8;
 constexpr int kThreads = 64 + kDequantWarps * 32;  // 320
 constexpr long long kDrainLimit = 1LL << 31;       // cycles (~1 s) for draining on abort
@@ -45,11 +48,15 @@ struct Cfg {
   static constexpr int kBBytes = BN * BK * 2;               // 16/32 KB
   static constexpr int kRawRow = BK * BITS / 8;             // 32 or 64 bytes
   static constexpr int kRawBytes = BN * kRawRow;
-  static constexpr int kStageTx = kABytes + kRawBytes;      // bytes landed per stage
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kABytes;
   static constexpr int kOffRaw = kOffB + kStages * kBBytes;
-  static constexpr int kOffBar = kOffRaw + kStages * kRawBytes;
+  static constexpr int kOffScale = kOffRaw + kStages * kRawBytes;
+  // either per-thread slots (kWinStages per job) or the whole [BN, K/32] tile (K <= 4096)
+  static constexpr int kScaleBytes = (kWinStages * (BN * 2) * 2 > BN * kTmaScaleCols * 2)
+                                         ? kWinStages * (BN * 2) * 2
+                                         : BN * kTmaScaleCols * 2;
+  static constexpr int kOffBar = (kOffScale + kScaleBytes + 15) & ~15;
   static constexpr int kSmem = kOffBar + 256 + 1024;        // barriers + alignment slack
   static constexpr uint32_t kTmemCols = BN;                 // power of two >= 32
   // Instruction descriptor: D f32, A/B bf16, both K-major, N = BN, M = 128.
@@ -65,10 +72,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 struct Shared {
-  uint64_t full[kStages];   // X tile + raw weight tile landed (TMA bytes)
+  uint64_t wfull[kStages];  // raw weight tile landed (TMA bytes)
+  uint64_t afull[kStages];  // bf16 X tile landed (TMA bytes)
   uint64_t bfull[kStages];  // bf16 weight tile written by the dequantisers
   uint64_t empty[kStages];  // MMAs reading the stage completed
   uint64_t acc_full;        // all MMAs of the tile completed
+  uint64_t sfull;           // scale tile landed (TMA bytes)
   uint64_t never;           // nothing arrives here: target of the injected stuck wait
   uint32_t tmem_base;
   int abort;
@@ -132,13 +141,15 @@ __device__ __forceinline__ uint4 dequant_int8_words(uint32_t w0, uint32_t w1, fl
 template <int BITS, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                    const uint16_t *__restrict__ scales, float *__restrict__ Y, int M, int N, int K,
+                    const __grid_constant__ CUtensorMap tm_s, const uint16_t *__restrict__ scales,
+                    float *__restrict__ Y, int M, int N, int K, int scales_tma,
                     long long wait_limit, long long stuck_wait) {
   using C = Cfg<BITS, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   Shared &sh = *reinterpret_cast<Shared *>(smem + C::kOffBar);
+  uint16_t *ssc = reinterpret_cast<uint16_t *>(smem + C::kOffScale);  // per-thread scale slots
   volatile int *abort = &sh.abort;
 
   const int warp = threadIdx.x >> 5;
@@ -146,14 +157,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n0 = blockIdx.x * BN;
   const int m0 = blockIdx.y * BM;
   const int num_k = (K + BK - 1) / BK;
+  const int pro = num_k < kStages ? num_k : kStages;  // stages issued before the PDL wait
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&sh.full[s], 1);
+      ptx::mbar_init(&sh.wfull[s], 1);
+      ptx::mbar_init(&sh.afull[s], 1);
       ptx::mbar_init(&sh.bfull[s], kDequantWarps * 32);
       ptx::mbar_init(&sh.empty[s], 1);
     }
     ptx::mbar_init(&sh.acc_full, 1);
+    ptx::mbar_init(&sh.sfull, 1);
     ptx::mbar_init(&sh.never, 1);
     sh.abort = 0;
     ptx::fence_mbar_init();
@@ -161,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tm_x);
     ptx::prefetch_tmap(&tm_w);
+    if (scales_tma) ptx::prefetch_tmap(&tm_s);
   }
   if (warp == 1) {
     ptx::tmem_alloc(&sh.tmem_base, C::kTmemCols);
@@ -171,26 +186,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  // X (written by the conversion kernel just before) and Y are touched only after this.
-  ptx::pdl_wait();
-
-  int issued = 0;  // producer: stages whose copies were issued
+  // Only X (produced by the conversion kernel) and Y depend on preceding kernels; the
+  // weight copies, the scale window and the first dequantisations run before the wait.
+  int issued_w = 0, issued_a = 0;  // producer: stages whose copies were issued
   bool mma_issued = false;
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int ks = 0; ks < num_k; ++ks) {
+      if (scales_tma) {
+        ptx::mbar_arrive_expect_tx(&sh.sfull, static_cast<uint32_t>(BN * (K >> 5) * 2));
+        ptx::tma_load_2d(ssc, &tm_s, &sh.sfull, 0, n0);
+      }
+      for (int ks = 0; ks < pro; ++ks) {
+        ptx::mbar_arrive_expect_tx(&sh.wfull[ks], C::kRawBytes);
+        ptx::tma_load_2d(smem + C::kOffRaw + ks * C::kRawBytes, &tm_w, &sh.wfull[ks],
+                         ks * C::kRawRow, n0);
+      }
+      issued_w = pro;
+      ptx::pdl_wait();
+      for (int ks = 0; ks < pro; ++ks) {
+        ptx::mbar_arrive_expect_tx(&sh.afull[ks], C::kABytes);
+        ptx::tma_load_2d(smem + C::kOffA + ks * C::kABytes, &tm_x, &sh.afull[ks], ks * BK, m0);
+      }
+      issued_a = pro;
+      for (int ks = pro; ks < num_k; ++ks) {
         const int s = ks % kStages;
         const uint32_t ph = (ks / kStages) & 1;
         if (!ptx::mbar_wait_bounded(&sh.empty[s], ph ^ 1, wait_limit, abort)) {
           record_timeout(abort);
           break;
         }
-        ptx::mbar_arrive_expect_tx(&sh.full[s], C::kStageTx);
-        ptx::tma_load_2d(smem + C::kOffA + s * C::kABytes, &tm_x, &sh.full[s], ks * BK, m0);
-        ptx::tma_load_2d(smem + C::kOffRaw + s * C::kRawBytes, &tm_w, &sh.full[s],
+        ptx::mbar_arrive_expect_tx(&sh.wfull[s], C::kRawBytes);
+        ptx::tma_load_2d(smem + C::kOffRaw + s * C::kRawBytes, &tm_w, &sh.wfull[s],
                          ks * C::kRawRow, n0);
-        issued = ks + 1;
+        issued_w = ks + 1;
+        ptx::mbar_arrive_expect_tx(&sh.afull[s], C::kABytes);
+        ptx::tma_load_2d(smem + C::kOffA + s * C::kABytes, &tm_x, &sh.afull[s], ks * BK, m0);
+        issued_a = ks + 1;
       }
     }
   } else if (warp == 1) {
@@ -204,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < num_k && ok; ++ks) {
         const int s = ks % kStages;
         const uint32_t ph = (ks / kStages) & 1;
-        ok = ptx::mbar_wait_bounded(&sh.full[s], ph, wait_limit, abort) &&
+        ok = ptx::mbar_wait_bounded(&sh.afull[s], ph, wait_limit, abort) &&
              ptx::mbar_wait_bounded(&sh.bfull[s], ph, wait_limit, abort);
         if (!ok) {
           record_timeout(abort);
@@ -228,23 +260,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = threadIdx.x - 64;  // 0 .. 255
     const int spr = K >> 5;
     constexpr int kJobs = BN * 2 / (kDequantWarps * 32);  // (row, half) jobs per thread
+    int wst0 = -kWinStages;                                // first stage of the loaded window
     bool ok = true;
+    if (scales_tma && !ptx::mbar_wait_bounded(&sh.sfull, 0, wait_limit, abort)) {
+      record_timeout(abort);
+      ok = false;
+    }
     for (int ks = 0; ks < num_k && ok; ++ks) {
       const int s = ks % kStages;
       const uint32_t ph = (ks / kStages) & 1;
-      // Scales for this stage (global loads issued before the wait).
-      float sv[kJobs];
+      if (!scales_tma && ks >= wst0 + kWinStages) {
+        // This thread's own scales for the next kWinStages stages, into its private slots
+        // of shared memory (only it reads them, so no barrier is involved). Rows past N and
+        // blocks past K/32 read as zero.
+        wst0 = ks;
+#pragma unroll 4
+        for (int j = 0; j < kWinStages; ++j) {
 #pragma unroll
-      for (int j = 0; j < kJobs; ++j) {
-        const int job = t + j * kDequantWarps * 32;
-        const int row = job % BN, h = job / BN;
-        const int kb = ks * 2 + h;
-        const int gr = n0 + row;
-        sv[j] = (gr < N && kb < spr)
-                    ? __half2float(__ushort_as_half(__ldg(scales + static_cast<size_t>(gr) * spr + kb)))
-                    : 0.f;
+          for (int jj = 0; jj < kJobs; ++jj) {
+            const int job = t + jj * kDequantWarps * 32;
+            const int gr = n0 + job % BN, kb = 2 * (ks + j) + job / BN;
+            ssc[(j * kJobs + jj) * (kDequantWarps * 32) + t] =
+                (gr < N && kb < spr) ? __ldg(scales + static_cast<size_t>(gr) * spr + kb) : 0;
+          }
+        }
       }
-      if (!ptx::mbar_wait_bounded(&sh.full[s], ph, wait_limit, abort)) {
+      if (!ptx::mbar_wait_bounded(&sh.wfull[s], ph, wait_limit, abort)) {
         record_timeout(abort);
         ok = false;
         break;
@@ -255,11 +296,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < kJobs; ++j) {
         const int job = t + j * kDequantWarps * 32;
         const int row = job % BN, h = job / BN;  // h: which 32-element half of the stage
+        const float s0 = __half2float(__ushort_as_half(
+            scales_tma ? ssc[row * spr + 2 * ks + h]
+                       : ssc[((ks - wst0) * kJobs + j) * (kDequantWarps * 32) + t]));
         uint8_t *brow = btile + row * 128;
         const int sw = row & 7;
         if constexpr (BITS == 4) {
           const uint4 wq = *reinterpret_cast<const uint4 *>(raw + row * C::kRawRow + h * 16);
-          const float s0 = sv[j];
           const float sj[4] = {s0, s0 * 0.0625f, s0 * 0.00390625f, s0 * 0.000244140625f};
           const uint32_t ws[4] = {wq.x, wq.y, wq.z, wq.w};
 #pragma unroll
@@ -275,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) {
             const int chunk = h * 4 + i;
             *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) =
-                dequant_int8_words(ws[2 * i], ws[2 * i + 1], sv[j]);
+                dequant_int8_words(ws[2 * i], ws[2 * i + 1], s0);
           }
         }
       }
@@ -284,6 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- epilogue: TMEM -> registers -> Y ----
+    // Y may be read by a preceding kernel: write it only after that grid completed.
+    ptx::pdl_wait();
     // tcgen05.ld is warp-collective, so the whole warp decides together.
     const bool mine = ok && ptx::mbar_wait_bounded(&sh.acc_full, 0, wait_limit, abort) && !*abort;
     const bool go = __all_sync(0xffffffffu, mine);
@@ -323,8 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0 && *abort) {
     // Only the last issue to each stage can still be in flight.
     int no_abort = 0;
-    for (int ks = issued - 1; ks >= 0 && ks >= issued - kStages; --ks)
-      ptx::mbar_wait_bounded(&sh.full[ks % kStages], (ks / kStages) & 1, kDrainLimit, &no_abort);
+    for (int ks = issued_w - 1; ks >= 0 && ks >= issued_w - kStages; --ks)
+      ptx::mbar_wait_bounded(&sh.wfull[ks % kStages], (ks / kStages) & 1, kDrainLimit, &no_abort);
+    for (int ks = issued_a - 1; ks >= 0 && ks >= issued_a - kStages; --ks)
+      ptx::mbar_wait_bounded(&sh.afull[ks % kStages], (ks / kStages) & 1, kDrainLimit, &no_abort);
+    if (scales_tma) ptx::mbar_wait_bounded(&sh.sfull, 0, kDrainLimit, &no_abort);
   }
   if (warp == 1 && lane == 0 && *abort && mma_issued) {
     // acc_full was committed after the last MMA this thread issued.
@@ -406,7 +454,18 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   });
   if (attr_err != cudaSuccess) return WOQ_ECUDA;
 
-  CUtensorMap tm_x, tm_w;
+  CUtensorMap tm_x, tm_w, tm_s;
+  const int64_t spr = w.k / 32;
+  // The whole scale tile [BN, K/32] comes by TMA when its rows are 16-byte multiples and
+  // it fits the shared-memory slot; otherwise each dequantiser loads its own scales.
+  const int scales_tma = (spr % 8 == 0 && spr <= kTmaScaleCols) ? 1 : 0;
+  if (scales_tma) {
+    if (!make_map(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w.scales, spr, w.n,
+                  static_cast<uint32_t>(spr), BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return WOQ_ECUDA;
+  } else {
+    std::memset(&tm_s, 0, sizeof(tm_s));
+  }
   if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, BM,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return WOQ_ECUDA;
@@ -446,8 +505,9 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
     cfg.numAttrs = 1;
     const long long lim = g_wait_limit_cycles > 0 ? g_wait_limit_cycles : kDefaultWaitLimit;
     const long long stuck = g_wait_limit_cycles < 0 ? -g_wait_limit_cycles : 0;
-    if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, w.scales, Y, static_cast<int>(m),
-                           static_cast<int>(w.n), static_cast<int>(w.k), lim, stuck) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_s, w.scales, Y, static_cast<int>(m),
+                           static_cast<int>(w.n), static_cast<int>(w.k), scales_tma, lim,
+                           stuck) != cudaSuccess)
       return WOQ_ECUDA;
     count_launches(1);
   }

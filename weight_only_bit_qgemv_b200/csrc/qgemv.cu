@@ -18,6 +18,7 @@
 //     order (deterministic).
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <mutex>
 #include <unordered_map>
 
@@ -25,6 +26,9 @@
 #include "woq_internal.h"
 
 namespace woq {
+
+__device__ unsigned int g_gemv_timeout_flag = 0;
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -184,7 +188,38 @@ __device__ __forceinline__ void chunk_int8(const float4 *__restrict__ xs4, int u
   }
 }
 
+// Loads one batch of weight chunks: chunks cb + 32u + lane (u < U) of rows row0 .. row0+R-1.
+// Rows at or past n, and chunks at or past cpr, read as zero codes with zero scale.
+template <int BITS, int R, int U>
+__device__ __forceinline__ void load_batch(const uint8_t *__restrict__ packed,
+                                           const uint16_t *__restrict__ scales, int n, int cpr,
+                                           int spr, size_t row_bytes, int row0, int cb, int lane,
+                                           uint4 (&wv)[U][R], float (&sc)[U][R]) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int c = cb + 32 * u + lane;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int row = row0 + r;
+      if (c < cpr && row < n) {
+        wv[u][r] = ptx::ldg_stream_v4(packed + static_cast<size_t>(row) * row_bytes +
+                                      static_cast<size_t>(c) * 16);
+        sc[u][r] = half_bits_to_float(
+            __ldg(scales + static_cast<size_t>(row) * spr + (BITS == 4 ? c : (c >> 1))));
+      } else {
+        wv[u][r] = make_uint4(0u, 0u, 0u, 0u);
+        sc[u][r] = 0.f;
+      }
+    }
+  }
+}
+
 // grid.x: CTAs striding over units of R rows; grid.y: passes of MT x rows.
+//
+// The weights never depend on the preceding kernel, so each warp issues the loads of its
+// first batch before waiting on the preceding grid (programmatic dependent launch): their
+// DRAM latency overlaps that grid's tail and the staging of x. Afterwards every batch's
+// loads are issued one batch ahead of its arithmetic.
 template <int BITS, int MT, int R, int U>
 __global__ void __launch_bounds__(kThreads)
     gemv_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
@@ -195,6 +230,16 @@ __global__ void __launch_bounds__(kThreads)
   const int warp = tid >> 5;
   const int m0 = blockIdx.y * MT;
   const int units_row = k >> 2;
+  const int cpr = (k * BITS) >> 7;  // 16-byte chunks per weight row
+  const int spr = k >> 5;           // scales per row
+  const size_t row_bytes = static_cast<size_t>(k) * BITS / 8;
+  const int units = (n + R - 1) / R;
+  const int stride = gridDim.x * kWarps;
+  int unit = blockIdx.x * kWarps + warp;
+
+  uint4 wv[U][R];
+  float sc[U][R];
+  load_batch<BITS, R, U>(packed, scales, n, cpr, spr, row_bytes, unit * R, 0, lane, wv, sc);
 
   // Everything below reads x or writes y, which a preceding kernel may produce or read.
   ptx::pdl_wait();
@@ -223,12 +268,7 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   ptx::pdl_launch_dependents();
 
-  const int cpr = (k * BITS) >> 7;  // 16-byte chunks per weight row
-  const int spr = k >> 5;           // scales per row
-  const size_t row_bytes = static_cast<size_t>(k) * BITS / 8;
-  const int units = (n + R - 1) / R;
-
-  for (int unit = blockIdx.x * kWarps + warp; unit < units; unit += gridDim.x * kWarps) {
+  for (; unit < units; unit += stride) {
     const int row0 = unit * R;
     float acc[R][MT];
 #pragma unroll
@@ -237,25 +277,13 @@ __global__ void __launch_bounds__(kThreads)
       for (int mm = 0; mm < MT; ++mm) acc[r][mm] = 0.f;
 
     for (int cb = 0; cb < cpr; cb += 32 * U) {
-      uint4 wv[U][R];
-      float sc[U][R];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = cb + 32 * u + lane;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const int row = row0 + r;
-          if (c < cpr && row < n) {
-            wv[u][r] = ptx::ldg_stream_v4(packed + static_cast<size_t>(row) * row_bytes +
-                                          static_cast<size_t>(c) * 16);
-            sc[u][r] = half_bits_to_float(
-                __ldg(scales + static_cast<size_t>(row) * spr + (BITS == 4 ? c : (c >> 1))));
-          } else {
-            wv[u][r] = make_uint4(0u, 0u, 0u, 0u);
-            sc[u][r] = 0.f;
-          }
-        }
-      }
+      // Issue the next batch (rest of this row group, else the next unit) before computing.
+      const bool same = cb + 32 * U < cpr;
+      uint4 nwv[U][R];
+      float nsc[U][R];
+      load_batch<BITS, R, U>(packed, scales, n, cpr, spr, row_bytes,
+                             same ? row0 : (unit + stride) * R, same ? cb + 32 * U : 0, lane,
+                             nwv, nsc);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int c = cb + 32 * u + lane;
@@ -266,6 +294,13 @@ __global__ void __launch_bounds__(kThreads)
             chunk_int8<MT, R>(xs4, units_row, c, wv[u], sc[u], acc);
         }
       }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          wv[u][r] = nwv[u][r];
+          sc[u][r] = nsc[u][r];
+        }
     }
 
 #pragma unroll
@@ -290,6 +325,189 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Bulk-copy pipeline variant (the default when a tile of rows fits a shared-memory stage).
+//
+// A tile is TR = 8 * RW consecutive weight rows; its codes and its scales are each one
+// contiguous range of memory, so one producer lane streams a tile with two 1-D bulk copies
+// (cp.async.bulk) into a ring of shared-memory stages, completion counted in bytes on an
+// mbarrier. Eight compute warps each take RW rows of a tile: lane l reads chunks l, l+32, ...
+// of its rows from shared memory and runs the same exact FP32 arithmetic as above. Memory
+// parallelism is the ring depth, not registers; the producer never touches x or y, so it
+// issues its copies before the wait on the preceding grid and they overlap that grid. A
+// partial last tile is read straight from global memory by the compute warps.
+// ---------------------------------------------------------------------------------------
+
+constexpr int kBulkWarps = 8;
+constexpr int kBulkThreads = (kBulkWarps + 1) * 32;
+constexpr int kMaxStages = 8;
+constexpr int kBulkHeader = 256;  // mbarriers + abort flag (BulkShared, padded)
+constexpr long long kGemvWaitLimit = 1LL << 32;   // cycles (~2 s)
+constexpr long long kGemvDrainLimit = 1LL << 31;  // cycles (~1 s)
+
+struct BulkShared {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  int abort;
+};
+static_assert(sizeof(BulkShared) <= kBulkHeader, "header too small");
+
+__device__ __forceinline__ void gemv_record_timeout(volatile int *abort) {
+  *abort = 1;
+  atomicOr(&g_gemv_timeout_flag, 1u);
+}
+
+template <int BITS, int MT, int RW>
+__global__ void __launch_bounds__(kBulkThreads)
+    gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
+                     const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n,
+                     int k, int stages, int stage_bytes, int x_bytes) {
+  constexpr int TR = kBulkWarps * RW;
+  extern __shared__ __align__(128) uint8_t smem[];
+  BulkShared &sh = *reinterpret_cast<BulkShared *>(smem);
+  float4 *xs4 = reinterpret_cast<float4 *>(smem + kBulkHeader);
+  uint8_t *ring = smem + kBulkHeader + x_bytes;
+  volatile int *abort = &sh.abort;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int m0 = blockIdx.y * MT;
+  const int units_row = k >> 2;
+  const int cpr = (k * BITS) >> 7;
+  const int spr = k >> 5;
+  const size_t row_bytes = static_cast<size_t>(k) * BITS / 8;
+  const uint32_t code_bytes = static_cast<uint32_t>(TR * row_bytes);
+  const uint32_t scale_bytes = static_cast<uint32_t>(TR * spr * 2);
+  const int full_tiles = n / TR;
+  const int num_tiles = (n + TR - 1) / TR;
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(&sh.full[s], 1);
+      ptx::mbar_init(&sh.empty[s], kBulkWarps);
+    }
+    sh.abort = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kBulkWarps) {
+    // ---- producer: weights only, so no wait on the preceding grid ----
+    if (lane == 0) {
+      int issued = 0;
+      for (int tile = blockIdx.x, i = 0; tile < full_tiles; tile += gridDim.x, ++i) {
+        const int s = i % stages;
+        const int round = i / stages;
+        if (round > 0 && !ptx::mbar_wait_bounded(&sh.empty[s], (round - 1) & 1, kGemvWaitLimit, abort)) {
+          gemv_record_timeout(abort);
+          break;
+        }
+        if (*abort) break;
+        uint8_t *dst = ring + static_cast<size_t>(s) * stage_bytes;
+        ptx::mbar_arrive_expect_tx(&sh.full[s], code_bytes + scale_bytes);
+        ptx::bulk_load(dst, packed + static_cast<size_t>(tile) * code_bytes, code_bytes, &sh.full[s]);
+        ptx::bulk_load(dst + code_bytes, scales + static_cast<size_t>(tile) * TR * spr, scale_bytes,
+                       &sh.full[s]);
+        issued = i + 1;
+      }
+      if (*abort) {
+        int no_abort = 0;  // only the last issue to each stage can still be in flight
+        for (int i = issued - 1; i >= 0 && i >= issued - stages; --i)
+          ptx::mbar_wait_bounded(&sh.full[i % stages], (i / stages) & 1, kGemvDrainLimit, &no_abort);
+      }
+    }
+    return;
+  }
+
+  // ---- compute warps ----
+  ptx::pdl_wait();
+  const int groups = k >> 3;
+  for (int idx = tid; idx < MT * groups; idx += kBulkWarps * 32) {
+    const int mm = idx / groups;
+    const int g = idx - mm * groups;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (m0 + mm < m) {
+      const float4 *src = reinterpret_cast<const float4 *>(x + static_cast<size_t>(m0 + mm) * k) + 2 * g;
+      a = src[0];
+      b = src[1];
+    }
+    float4 pa = a, pb = b;
+    if constexpr (BITS == 4) {
+      pa = make_float4(a.x, b.x, a.y, b.y);
+      pb = make_float4(a.z, b.z, a.w, b.w);
+    }
+    float4 *row = xs4 + mm * units_row;
+    row[swz(2 * g)] = pa;
+    row[swz(2 * g + 1)] = pb;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kBulkWarps * 32) : "memory");
+  ptx::pdl_launch_dependents();
+
+  for (int tile = blockIdx.x, i = 0; tile < num_tiles; tile += gridDim.x, ++i) {
+    const bool staged = tile < full_tiles;
+    const int s = i % stages;
+    if (staged && !ptx::mbar_wait_bounded(&sh.full[s], (i / stages) & 1, kGemvWaitLimit, abort)) {
+      gemv_record_timeout(abort);
+      break;
+    }
+    const uint8_t *stage = ring + static_cast<size_t>(s) * stage_bytes;
+    const int lrow0 = warp * RW;  // this warp's first row within the tile
+    const int row0 = tile * TR + lrow0;
+    float acc[RW][MT];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = 0.f;
+
+    for (int c = lane; c < cpr; c += 32) {
+      const int blk = BITS == 4 ? c : (c >> 1);
+      uint4 wv[RW];
+      float sc[RW];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        if (staged) {
+          wv[r] = *reinterpret_cast<const uint4 *>(stage + (lrow0 + r) * row_bytes + c * 16);
+          sc[r] = half_bits_to_float(
+              reinterpret_cast<const uint16_t *>(stage + code_bytes)[(lrow0 + r) * spr + blk]);
+        } else if (row0 + r < n) {
+          wv[r] = ptx::ldg_stream_v4(packed + static_cast<size_t>(row0 + r) * row_bytes + c * 16);
+          sc[r] = half_bits_to_float(__ldg(scales + static_cast<size_t>(row0 + r) * spr + blk));
+        } else {
+          wv[r] = make_uint4(0u, 0u, 0u, 0u);
+          sc[r] = 0.f;
+        }
+      }
+      if constexpr (BITS == 4)
+        chunk_int4<MT, RW>(xs4, units_row, c, wv, sc, acc);
+      else
+        chunk_int8<MT, RW>(xs4, units_row, c, wv, sc, acc);
+    }
+    if (staged) {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.empty[s]);
+    }
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float v = acc[r][mm];
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        acc[r][mm] = v;
+      }
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm)
+        if (lane == r * MT + mm && row0 + r < n && m0 + mm < m)
+          y[static_cast<size_t>(m0 + mm) * n + row0 + r] = acc[r][mm];
+  }
+}
+
 struct OccKey {
   const void *fn;
   size_t smem;
@@ -306,7 +524,7 @@ struct OccHash {
 
 // Resident CTAs per SM for (kernel, dynamic smem) on the device; also raises the
 // kernel's dynamic shared memory limit when needed. Cached.
-int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev) {
+int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev, int threads = kThreads) {
   static std::mutex mu;
   static std::unordered_map<OccKey, int, OccHash> cache;
   const OccKey key{fn, smem, dev.device};
@@ -321,7 +539,7 @@ int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev) {
       return -1;
   }
   int nb = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem) != cudaSuccess)
     return -1;
   std::lock_guard<std::mutex> g(mu);
   cache[key] = nb;
@@ -382,6 +600,68 @@ int pick_ru(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
              : launch_t<BITS, MT, 1, 1>(x, m, w, y, s, dev, pdl);
 }
 
+// Bulk-pipeline launch. Returns 1 (not launched) when the shape does not suit it.
+constexpr size_t kStageTarget = 20 * 1024;   // bytes per ring stage to aim for
+constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
+
+template <int BITS, int MT, int RW>
+int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                  const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes) {
+  auto kern = gemv_bulk_kernel<BITS, MT, RW>;
+  constexpr int TR = kBulkWarps * RW;
+  const int64_t num_tiles = (w.n + TR - 1) / TR;
+  const int64_t full_tiles = w.n / TR;
+  // stages: enough for the tiles one CTA will see, within the smem budget
+  const int64_t want_grid = std::min<int64_t>(num_tiles, static_cast<int64_t>(dev.sm_count) * 2);
+  int64_t stages = want_grid > 0 ? (full_tiles + want_grid - 1) / want_grid : 1;
+  const int64_t fit = (static_cast<int64_t>(kCtaSmemBudget) - kBulkHeader - static_cast<int64_t>(x_bytes)) /
+                      static_cast<int64_t>(stage_bytes);
+  stages = std::max<int64_t>(1, std::min<int64_t>({stages, fit, kMaxStages}));
+  const size_t smem = kBulkHeader + x_bytes + stages * stage_bytes;
+  const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev, kBulkThreads);
+  if (nb <= 0) return WOQ_ECUDA;
+  const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(num_tiles, static_cast<int64_t>(dev.sm_count) * nb));
+  const int64_t gy = (m + MT - 1) / MT;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 1);
+  cfg.blockDim = dim3(kBulkThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, w.packed, w.scales, y, static_cast<int>(m),
+                                           static_cast<int>(w.n), static_cast<int>(w.k),
+                                           static_cast<int>(stages), static_cast<int>(stage_bytes),
+                                           static_cast<int>(x_bytes));
+  if (e != cudaSuccess) return WOQ_ECUDA;
+  count_launches(1);
+  return WOQ_OK;
+}
+
+template <int BITS, int MT>
+int try_bulk(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+             const DevInfo &dev, bool pdl) {
+  const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
+  const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
+  int rw = MT <= 2 ? 4 : 2;  // more rows per warp only where registers allow
+  while (rw > 1 && kBulkWarps * rw * row_total > kStageTarget) rw /= 2;
+  const size_t stage_bytes = (kBulkWarps * rw * row_total + 127) & ~size_t(127);
+  if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return 1;
+  if (w.n < kBulkWarps * rw) rw = 1;  // tiny n: one row per warp, all from global memory
+  if constexpr (MT <= 2) {
+    if (rw == 4) return launch_bulk_t<BITS, MT, 4>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+  }
+  switch (rw) {
+    case 2: return launch_bulk_t<BITS, MT, 2>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+    default: return launch_bulk_t<BITS, MT, 1>(x, m, w, y, s, dev, pdl,
+                                             (kBulkWarps * row_total + 127) & ~size_t(127), x_bytes);
+  }
+}
+
 template <int BITS>
 int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
             const DevInfo &dev, bool pdl) {
@@ -389,6 +669,14 @@ int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
   const size_t limit = dev.smem_optin < 200 * 1024 ? dev.smem_optin : 200 * 1024;
   while (mt > 1 && static_cast<size_t>(mt) * w.k * sizeof(float) > limit) mt /= 2;
   if (static_cast<size_t>(mt) * w.k * sizeof(float) > limit) return WOQ_ESHAPE;
+  int rc = 1;
+  switch (mt) {
+    case 1: rc = try_bulk<BITS, 1>(x, m, w, y, s, dev, pdl); break;
+    case 2: rc = try_bulk<BITS, 2>(x, m, w, y, s, dev, pdl); break;
+    case 4: rc = try_bulk<BITS, 4>(x, m, w, y, s, dev, pdl); break;
+    default: rc = try_bulk<BITS, 8>(x, m, w, y, s, dev, pdl); break;
+  }
+  if (rc != 1) return rc;
   switch (mt) {
     case 1: return pick_ru<BITS, 1>(x, m, w, y, s, dev, pdl);
     case 2: return pick_ru<BITS, 2>(x, m, w, y, s, dev, pdl);
@@ -398,6 +686,17 @@ int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
 }
 
 }  // namespace
+
+int read_gemv_timeout_flag(int clear, unsigned *value) {
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gemv_timeout_flag, sizeof(v)) != cudaSuccess) return WOQ_ECUDA;
+  if (clear && v) {
+    const unsigned z = 0;
+    if (cudaMemcpyToSymbol(g_gemv_timeout_flag, &z, sizeof(z)) != cudaSuccess) return WOQ_ECUDA;
+  }
+  *value = v;
+  return WOQ_OK;
+}
 
 int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                      const DevInfo &dev, bool pdl) {

@@ -30,6 +30,9 @@ void count_launches(uint64_t n);
 int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                      const DevInfo &dev, bool pdl);
 
+// Reads (and optionally clears) the GEMV kernels' record of bounded waits that gave up.
+int read_gemv_timeout_flag(int clear, unsigned *value);
+
 // ---- qgemm_tc.cu ----
 // Workspace bytes of the tensor-core path (the bf16 copy of X).
 size_t gemm_tc_workspace_bytes(int64_t m, int64_t k);
