@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&sh.wfull[s], 1);
       ptx::mbar_init(&sh.afull[s], 1);
-      ptx::mbar_init(&sh.bfull[s], kDequantWarps * 32);
+      ptx::mbar_init(&sh.bfull[s], kDequantWarps);  // one elected arrival per warp
       ptx::mbar_init(&sh.empty[s], 1);
     }
     ptx::mbar_init(&sh.acc_full, 1);
@@ -262,7 +262,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kJobs = BN * 2 / (kDequantWarps * 32);  // (row, half) jobs per thread
     int wst0 = -kWinStages;                                // first stage of the loaded window
     bool ok = true;
-    if (scales_tma && !ptx::mbar_wait_bounded(&sh.sfull, 0, wait_limit, abort)) {
+    // Wait outcomes are made warp-uniform: the loop below contains warp-collective steps.
+    if (scales_tma &&
+        !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.sfull, 0, wait_limit, abort))) {
       record_timeout(abort);
       ok = false;
     }
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ptx::mbar_wait_bounded(&sh.wfull[s], ph, wait_limit, abort)) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.wfull[s], ph, wait_limit, abort))) {
         record_timeout(abort);
         ok = false;
         break;
@@ -322,8 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // Each lane makes its tile writes visible to the async proxy (the tensor core), the
+      // warp converges, and one lane arrives for the warp.
       ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(&sh.bfull[s]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.bfull[s]);
     }
 
     // ---- epilogue: TMEM -> registers -> Y ----

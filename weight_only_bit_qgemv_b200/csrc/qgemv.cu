@@ -188,6 +188,96 @@ __device__ __forceinline__ void chunk_int8(const float4 *__restrict__ xs4, int u
   }
 }
 
+// int8: one whole block (32 codes = chunks 2b and 2b+1, x units 8b .. 8b+7) of R rows
+// against MT x rows; one scale per row, applied once to the block sum.
+template <int MT, int R>
+__device__ __forceinline__ void block_int8(const float4 *__restrict__ xs4, int units_row, int b,
+                                           const uint4 (&lo)[R], const uint4 (&hi)[R],
+                                           const float (&sc)[R], float (&acc)[R][MT]) {
+  if constexpr (MT <= 2) {
+    float4 xv[MT][8];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) xv[mm][t] = xs4[mm * units_row + swz(8 * b + t)];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 a2[MT];
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) a2[mm] = make_float2(0.f, 0.f);
+      const uint32_t ws[8] = {lo[r].x, lo[r].y, lo[r].z, lo[r].w, hi[r].x, hi[r].y, hi[r].z, hi[r].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float2 p[2];
+        unpack_int8_word(ws[i], p);
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          a2[mm] = __ffma2_rn(p[0], make_float2(xv[mm][i].x, xv[mm][i].y), a2[mm]);
+          a2[mm] = __ffma2_rn(p[1], make_float2(xv[mm][i].z, xv[mm][i].w), a2[mm]);
+        }
+      }
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], a2[mm].x + a2[mm].y, acc[r][mm]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 p[8][2];
+      const uint32_t ws[8] = {lo[r].x, lo[r].y, lo[r].z, lo[r].w, hi[r].x, hi[r].y, hi[r].z, hi[r].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) unpack_int8_word(ws[i], p[i]);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 xa = xs4[mm * units_row + swz(8 * b + i)];
+          a2 = __ffma2_rn(p[i][0], make_float2(xa.x, xa.y), a2);
+          a2 = __ffma2_rn(p[i][1], make_float2(xa.z, xa.w), a2);
+        }
+        acc[r][mm] = fmaf(sc[r], a2.x + a2.y, acc[r][mm]);
+      }
+    }
+  }
+}
+
+// Dot products of RW consecutive weight rows with MT staged x rows, lane l taking blocks
+// l, l+32, ... . SMEM: rows come from a shared-memory stage (all RW rows present);
+// otherwise from global memory, rows at or past `valid` reading as zero.
+template <int BITS, int MT, int RW, bool SMEM>
+__device__ __forceinline__ void rows_dot(const float4 *__restrict__ xs4, int units_row, int spr,
+                                         int lane, const uint8_t *codes, size_t row_stride,
+                                         const uint16_t *scs, int valid, float (&acc)[RW][MT]) {
+  constexpr int kBlockBytes = BITS * 4;  // 16 (int4) or 32 (int8)
+  for (int b = lane; b < spr; b += 32) {
+    uint4 lo[RW], hi[RW];
+    float sc[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      const uint8_t *pr = codes + r * row_stride + b * kBlockBytes;
+      if (SMEM || r < valid) {
+        if constexpr (SMEM) {
+          lo[r] = *reinterpret_cast<const uint4 *>(pr);
+          if constexpr (BITS == 8) hi[r] = *reinterpret_cast<const uint4 *>(pr + 16);
+          sc[r] = half_bits_to_float(scs[r * spr + b]);
+        } else {
+          lo[r] = ptx::ldg_stream_v4(pr);
+          if constexpr (BITS == 8) hi[r] = ptx::ldg_stream_v4(pr + 16);
+          sc[r] = half_bits_to_float(__ldg(scs + r * spr + b));
+        }
+      } else {
+        lo[r] = make_uint4(0u, 0u, 0u, 0u);
+        hi[r] = lo[r];
+        sc[r] = 0.f;
+      }
+    }
+    if constexpr (BITS == 4)
+      chunk_int4<MT, RW>(xs4, units_row, b, lo, sc, acc);
+    else
+      block_int8<MT, RW>(xs4, units_row, b, lo, hi, sc, acc);
+  }
+}
+
 // Loads one batch of weight chunks: chunks cb + 32u + lane (u < U) of rows row0 .. row0+R-1.
 // Rows at or past n, and chunks at or past cpr, read as zero codes with zero scale.
 template <int BITS, int R, int U>
@@ -447,7 +537,9 @@ __global__ void __launch_bounds__(kBulkThreads)
   for (int tile = blockIdx.x, i = 0; tile < num_tiles; tile += gridDim.x, ++i) {
     const bool staged = tile < full_tiles;
     const int s = i % stages;
-    if (staged && !ptx::mbar_wait_bounded(&sh.full[s], (i / stages) & 1, kGemvWaitLimit, abort)) {
+    // The outcome is made warp-uniform: shuffles and the elected arrival follow.
+    if (staged && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.full[s], (i / stages) & 1,
+                                                                   kGemvWaitLimit, abort))) {
       gemv_record_timeout(abort);
       break;
     }
@@ -460,28 +552,14 @@ __global__ void __launch_bounds__(kBulkThreads)
 #pragma unroll
       for (int mm = 0; mm < MT; ++mm) acc[r][mm] = 0.f;
 
-    for (int c = lane; c < cpr; c += 32) {
-      const int blk = BITS == 4 ? c : (c >> 1);
-      uint4 wv[RW];
-      float sc[RW];
-#pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        if (staged) {
-          wv[r] = *reinterpret_cast<const uint4 *>(stage + (lrow0 + r) * row_bytes + c * 16);
-          sc[r] = half_bits_to_float(
-              reinterpret_cast<const uint16_t *>(stage + code_bytes)[(lrow0 + r) * spr + blk]);
-        } else if (row0 + r < n) {
-          wv[r] = ptx::ldg_stream_v4(packed + static_cast<size_t>(row0 + r) * row_bytes + c * 16);
-          sc[r] = half_bits_to_float(__ldg(scales + static_cast<size_t>(row0 + r) * spr + blk));
-        } else {
-          wv[r] = make_uint4(0u, 0u, 0u, 0u);
-          sc[r] = 0.f;
-        }
-      }
-      if constexpr (BITS == 4)
-        chunk_int4<MT, RW>(xs4, units_row, c, wv, sc, acc);
-      else
-        chunk_int8<MT, RW>(xs4, units_row, c, wv, sc, acc);
+    if (staged) {
+      rows_dot<BITS, MT, RW, true>(xs4, units_row, spr, lane, stage + lrow0 * row_bytes, row_bytes,
+                                   reinterpret_cast<const uint16_t *>(stage + code_bytes) + lrow0 * spr,
+                                   RW, acc);
+    } else {
+      rows_dot<BITS, MT, RW, false>(xs4, units_row, spr, lane,
+                                    packed + static_cast<size_t>(row0) * row_bytes, row_bytes,
+                                    scales + static_cast<size_t>(row0) * spr, n - row0, acc);
     }
     if (staged) {
       __syncwarp();
