@@ -3,6 +3,7 @@
 // synchronises a stream (woq_device_status excepted, which exists to synchronise).
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "woq.h"
@@ -78,6 +79,13 @@ int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream
   return woq::launch_gemv_fp32(x, m, *w, y, static_cast<cudaStream_t>(stream), dev, true);
 }
 
+// SM count the tensor-core plan is made for: the current device's, or 0 (no K-splits) when
+// no device can be queried, so that sizing never fails.
+static int plan_sm_count() {
+  DevInfo dev;
+  return woq::current_device(&dev) == WOQ_OK ? dev.sm_count : 0;
+}
+
 static int resolve_path(int32_t path, int64_t m) {
   if (path == WOQ_PATH_AUTO) return m >= 128 ? WOQ_PATH_BF16_TC : WOQ_PATH_FP32;
   return path;
@@ -86,7 +94,8 @@ static int resolve_path(int32_t path, int64_t m) {
 size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path) {
   if (woq::check_weight(w) != WOQ_OK || m < 1) return 0;
   if (path != WOQ_PATH_AUTO && path != WOQ_PATH_FP32 && path != WOQ_PATH_BF16_TC) return 0;
-  return resolve_path(path, m) == WOQ_PATH_BF16_TC ? woq::gemm_tc_workspace_bytes(m, w->k) : 0;
+  if (resolve_path(path, m) != WOQ_PATH_BF16_TC) return 0;
+  return woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX).total;
 }
 
 int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path,
@@ -99,9 +108,10 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
   if (!woq::aligned(X, 16) || !woq::aligned(Y, 16)) return WOQ_EALIGN;
   const int p = resolve_path(path, m);
   if (p == WOQ_PATH_FP32 && w->k > 32768) return WOQ_ESHAPE;
+  woq::GemmPlan plan;
   if (p == WOQ_PATH_BF16_TC) {
-    const size_t need = woq::gemm_tc_workspace_bytes(m, w->k);
-    if (!workspace || workspace_bytes < need) return WOQ_EWORKSPACE;
+    plan = woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX);
+    if (!workspace || workspace_bytes < plan.total) return WOQ_EWORKSPACE;
     if (!woq::aligned(workspace, 256)) return WOQ_EALIGN;
   }
   DevInfo dev;
@@ -109,7 +119,7 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
   if (rc != WOQ_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (p == WOQ_PATH_FP32) return woq::launch_gemv_fp32(X, m, *w, Y, s, dev, true);
-  return woq::launch_gemm_tc(X, m, *w, Y, workspace, s, dev);
+  return woq::launch_gemm_tc(X, m, *w, Y, workspace, plan, s, dev);
 }
 
 int woq_device_status(int clear) {

@@ -60,13 +60,15 @@ extern "C" int qgemm_bf16_noalloc(const float *X, int64_t m, const woq_weight *w
   if ((reinterpret_cast<uintptr_t>(w->packed) & 63) || (reinterpret_cast<uintptr_t>(w->scales) & 63))
     return WOQ_EALIGN;
   if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(Y) & 15)) return WOQ_EALIGN;
-  // The bf16 copy of X must fit in the fixed scratch array.
-  if (woq::gemm_tc_workspace_bytes(m, w->k) > woq::kScratchBytes) return WOQ_ESHAPE;
+  // The bf16 copy of X must fit in the fixed scratch array (K-split partials are used only
+  // as far as the rest of it allows).
+  if (woq::plan_gemm_tc(m, w->n, w->k, 0, woq::kScratchBytes).xb > woq::kScratchBytes) return WOQ_ESHAPE;
   woq::DevInfo dev;
   int rc = woq::current_device(&dev);
   if (rc != WOQ_OK) return rc;
   void *scratch = nullptr;
   rc = woq::scratch_address(dev.device, &scratch);
   if (rc != WOQ_OK) return rc;
-  return woq::launch_gemm_tc(X, m, *w, Y, scratch, static_cast<cudaStream_t>(stream), dev);
+  const woq::GemmPlan plan = woq::plan_gemm_tc(m, w->n, w->k, dev.sm_count, woq::kScratchBytes);
+  return woq::launch_gemm_tc(X, m, *w, Y, scratch, plan, static_cast<cudaStream_t>(stream), dev);
 }

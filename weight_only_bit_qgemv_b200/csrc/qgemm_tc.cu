@@ -1,23 +1,27 @@
 // tcgen05 qgemm (prefill): Y[m, n] = bf16(X) . bf16(W_hat)^T with FP32 accumulation in
 // tensor memory. "TinyMOSS-Diarize", "How we built it": the prefill GEMM unpacks each
 // weight group once into an on-chip tile and reuses it across all activation rows; here
-// the tile is dequantised once into shared memory per (N-tile, K-stage) and is read by the
-// tensor core for all 128 rows of the M-tile.
+// each weight tile is dequantised once into shared memory per (output tile, K-stage) and
+// read by the tensor core for all 128 rows of the M-tile.
 //
-// Per CTA: one 128 x BN output tile, K in stages of 64.
-//   warp 0        producer: bulk tensor copies (TMA) of the bf16 X tile (128B-swizzled) and
-//                 of the raw packed weight tile, one mbarrier per stage (byte counted)
-//   warp 1        TMEM allocation; one elected thread issues tcgen05.mma (M=128, N=BN,
-//                 K=16, bf16 x bf16 -> f32) and commits completions to mbarriers
-//   warps 2..9    dequantisers: raw codes + binary16 scales -> bf16(scale * code) written in
-//                 the 128B-swizzled K-major layout the MMA descriptor names; afterwards the
-//                 same warps drain the accumulator (tcgen05.ld) and store FP32 Y
-// Every mbarrier wait is bounded; a wait that gives up records the event in a device flag,
-// makes the CTA's other roles stop, drains the copies and MMAs already issued, frees TMEM
-// and returns.
+// Persistent, warp-specialised kernel; one CTA per SM walks 128 x 128 output tiles.
+//   warp 0        producer: bulk tensor copies (TMA, no multicast) of the bf16 X tile
+//                 (128B-swizzled) and the raw code tile into a ring of SL load stages, and
+//                 of each output tile's [128, K/32] scale tile into a double buffer
+//   warp 1        TMEM owner; one thread issues tcgen05.mma (M=128, N=128, K=16, bf16 x
+//                 bf16 -> f32) into one of two accumulators and commits completions
+//   warps 2..9    dequantisers: raw codes + binary16 scales -> bf16(scale * code) written
+//                 into a short ring of B tiles in the 128B-swizzled K-major layout that the
+//                 MMA's shared-memory descriptor names
+//   warps 10..13  epilogue: tcgen05.ld of the finished accumulator -> FP32 Y, while the MMA
+//                 thread already fills the other accumulator with the next tile
+// Every mbarrier wait is bounded. A wait that gives up records the event in a device flag
+// and stops the CTA's other roles; the CTA drains the copies and MMAs it issued, frees
+// tensor memory and returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -31,57 +35,64 @@ __device__ unsigned int g_wait_timeout_flag = 0;
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 64;           // bf16 elements per stage = one 128-byte swizzle row
-constexpr int kStages = 4;
-constexpr int kWinStages = 32;   // K-stages whose scales each dequantiser holds in shared memory
-constexpr int kTmaScaleCols = 128;  // scale tile copied whole by TMA when K/32 <= this
-constexpr int kDequantWarps = 8;
-constexpr int kThreads = 64 + kDequantWarps * 32;  // 320
-constexpr long long kDrainLimit = 1LL << 31;       // cycles (~1 s) for draining on abort
-constexpr long long kDefaultWaitLimit = 1LL << 32;  // cycles (~2 s) for ordinary waits
+constexpr int BK = 64;              // bf16 elements per stage = one 128-byte swizzle row
+constexpr int kMaxSL = 8;           // load stages (X tile + raw code tile)
+constexpr int kSB = 2;              // dequantised B tiles
+constexpr int kTmaScaleCols = 128;  // scale tile copied by TMA when K/32 <= this (and % 8 == 0)
+constexpr int kDequantWarps = 16;  // four per scheduler: each warp's chain is latency-bound
+constexpr int kDequantThreads = kDequantWarps * 32;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = (2 + kDequantWarps + kEpiWarps) * 32;  // 704
+constexpr int kABytes = BM * BK * 2;                            // 16 KB
+constexpr long long kDrainLimit = 1LL << 31;                    // cycles (~1 s)
+constexpr long long kDefaultWaitLimit = 1LL << 32;              // cycles (~2 s)
+constexpr int kSmemMax = 227 * 1024;
+
+// Instruction descriptor: D f32, A/B bf16, both K-major, N = bn, M = BM.
+__host__ __device__ constexpr uint32_t idesc_for(int bn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) |
+         (static_cast<uint32_t>(BM >> 4) << 24);
+}
 
 long long g_wait_limit_cycles = 0;  // test hook: > 0 wait limit, < 0 inject a stuck wait
 
-template <int BITS, int BN>
-struct Cfg {
-  static constexpr int kABytes = BM * BK * 2;               // 16 KB
-  static constexpr int kBBytes = BN * BK * 2;               // 16/32 KB
-  static constexpr int kRawRow = BK * BITS / 8;             // 32 or 64 bytes
-  static constexpr int kRawBytes = BN * kRawRow;
-  static constexpr int kOffA = 0;
-  static constexpr int kOffB = kOffA + kStages * kABytes;
-  static constexpr int kOffRaw = kOffB + kStages * kBBytes;
-  static constexpr int kOffScale = kOffRaw + kStages * kRawBytes;
-  // either per-thread slots (kWinStages per job) or the whole [BN, K/32] tile (K <= 4096)
-  static constexpr int kScaleBytes = (kWinStages * (BN * 2) * 2 > BN * kTmaScaleCols * 2)
-                                         ? kWinStages * (BN * 2) * 2
-                                         : BN * kTmaScaleCols * 2;
-  static constexpr int kOffBar = (kOffScale + kScaleBytes + 15) & ~15;
-  static constexpr int kSmem = kOffBar + 256 + 1024;        // barriers + alignment slack
-  static constexpr uint32_t kTmemCols = BN;                 // power of two >= 32
-  // Instruction descriptor: D f32, A/B bf16, both K-major, N = BN, M = 128.
-  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                     (static_cast<uint32_t>(BN >> 3) << 17) |
-                                     (static_cast<uint32_t>(BM >> 4) << 24);
+struct Shared {
+  uint64_t afull[kMaxSL];   // X tile landed (TMA bytes)
+  uint64_t wfull[kMaxSL];   // raw code tile landed (TMA bytes)
+  uint64_t lempty[kMaxSL];  // load stage free: MMA commit + one arrival per dequant warp
+  uint64_t bfull[kSB];      // B tile written (one arrival per dequant warp)
+  uint64_t bempty[kSB];     // B tile read by the MMAs (commit)
+  uint64_t sfull[2];        // scale tile landed (TMA bytes)
+  uint64_t sempty[2];       // scale tile done with (one arrival per dequant warp)
+  uint64_t accfull[2];      // accumulator complete (commit)
+  uint64_t accempty[2];     // accumulator drained (one arrival per epilogue warp)
+  uint64_t never;           // nothing arrives here: target of the injected stuck wait
+  uint64_t drain;           // MMA completion on abort
+  uint32_t tmem_base;
+  int abort;
 };
+
+// Shared-memory layout for a given number of load stages and scale-tile size.
+struct Layout {
+  int a, b, raw, sc, bar, total;
+};
+__host__ __device__ inline Layout make_layout(int bits, int bn, int sl, int sc_bytes, int sc_bufs) {
+  Layout L;
+  const int raw_bytes = bn * BK * bits / 8;
+  L.a = 0;
+  L.b = L.a + sl * kABytes;
+  L.raw = L.b + kSB * bn * BK * 2;
+  L.sc = L.raw + sl * raw_bytes;
+  L.bar = (L.sc + sc_bufs * sc_bytes + 127) & ~127;
+  L.total = L.bar + static_cast<int>(sizeof(Shared)) + 1024;  // + base alignment slack
+  return L;
+}
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (1ull << 16) | (64ull << 32) |
          (1ull << 46) | (2ull << 61);
 }
-
-struct Shared {
-  uint64_t wfull[kStages];  // raw weight tile landed (TMA bytes)
-  uint64_t afull[kStages];  // bf16 X tile landed (TMA bytes)
-  uint64_t bfull[kStages];  // bf16 weight tile written by the dequantisers
-  uint64_t empty[kStages];  // MMAs reading the stage completed
-  uint64_t acc_full;        // all MMAs of the tile completed
-  uint64_t sfull;           // scale tile landed (TMA bytes)
-  uint64_t never;           // nothing arrives here: target of the injected stuck wait
-  uint32_t tmem_base;
-  int abort;
-};
 
 __device__ __forceinline__ void record_timeout(volatile int *abort) {
   *abort = 1;
@@ -142,43 +153,59 @@ template <int BITS, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s, const uint16_t *__restrict__ scales,
-                    float *__restrict__ Y, int M, int N, int K, int scales_tma,
-                    long long wait_limit, long long stuck_wait) {
-  using C = Cfg<BITS, BN>;
+                    float *__restrict__ Y, int M, int N, int K, int sl_stages, int sc_bytes,
+                    int sc_bufs, int splits, float *__restrict__ partials, long long wait_limit,
+                    long long stuck_wait) {
+  constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
+  constexpr int kRawBytes = BN * kRawRow;
+  constexpr int kBBytes = BN * BK * 2;
+  constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+  constexpr uint32_t kIdesc = idesc_for(BN);
+  const Layout L = make_layout(BITS, BN, sl_stages, sc_bytes, sc_bufs);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  Shared &sh = *reinterpret_cast<Shared *>(smem + C::kOffBar);
-  uint16_t *ssc = reinterpret_cast<uint16_t *>(smem + C::kOffScale);  // per-thread scale slots
+  Shared &sh = *reinterpret_cast<Shared *>(smem + L.bar);
   volatile int *abort = &sh.abort;
+  const bool sc_tma = sc_bytes > 0;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * BM;
   const int num_k = (K + BK - 1) / BK;
-  const int pro = num_k < kStages ? num_k : kStages;  // stages issued before the PDL wait
+  const int num_m = (M + BM - 1) / BM;
+  // Work unit u covers output tile u / splits and K-stages [ks0, ks1) of split u % splits.
+  const int num_units = num_m * ((N + BN - 1) / BN) * splits;
+  const int kps = (num_k + splits - 1) / splits;
+  const int SL = sl_stages;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(&sh.wfull[s], 1);
+    for (int s = 0; s < SL; ++s) {
       ptx::mbar_init(&sh.afull[s], 1);
-      ptx::mbar_init(&sh.bfull[s], kDequantWarps);  // one elected arrival per warp
-      ptx::mbar_init(&sh.empty[s], 1);
+      ptx::mbar_init(&sh.wfull[s], 1);
+      ptx::mbar_init(&sh.lempty[s], 1 + kDequantWarps);  // MMA commit + dequant warps
     }
-    ptx::mbar_init(&sh.acc_full, 1);
-    ptx::mbar_init(&sh.sfull, 1);
+    for (int s = 0; s < kSB; ++s) {
+      ptx::mbar_init(&sh.bfull[s], kDequantWarps);
+      ptx::mbar_init(&sh.bempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&sh.sfull[s], 1);
+      ptx::mbar_init(&sh.sempty[s], kDequantWarps);
+      ptx::mbar_init(&sh.accfull[s], 1);
+      ptx::mbar_init(&sh.accempty[s], kEpiWarps);
+    }
     ptx::mbar_init(&sh.never, 1);
+    ptx::mbar_init(&sh.drain, 1);
     sh.abort = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tm_x);
     ptx::prefetch_tmap(&tm_w);
-    if (scales_tma) ptx::prefetch_tmap(&tm_s);
+    if (sc_tma) ptx::prefetch_tmap(&tm_s);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&sh.tmem_base, C::kTmemCols);
+    ptx::tmem_alloc(&sh.tmem_base, kTmemCols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -186,46 +213,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  // Only X (produced by the conversion kernel) and Y depend on preceding kernels; the
-  // weight copies, the scale window and the first dequantisations run before the wait.
-  int issued_w = 0, issued_a = 0;  // producer: stages whose copies were issued
+  int issued_w = 0, issued_a = 0, issued_s = 0;  // producer bookkeeping for the drain
   bool mma_issued = false;
 
   if (warp == 0) {
+    // ---- producer (one lane). Only X depends on preceding kernels: wait before it. ----
     if (lane == 0) {
-      if (scales_tma) {
-        ptx::mbar_arrive_expect_tx(&sh.sfull, static_cast<uint32_t>(BN * (K >> 5) * 2));
-        ptx::tma_load_2d(ssc, &tm_s, &sh.sfull, 0, n0);
-      }
-      for (int ks = 0; ks < pro; ++ks) {
-        ptx::mbar_arrive_expect_tx(&sh.wfull[ks], C::kRawBytes);
-        ptx::tma_load_2d(smem + C::kOffRaw + ks * C::kRawBytes, &tm_w, &sh.wfull[ks],
-                         ks * C::kRawRow, n0);
-      }
-      issued_w = pro;
-      ptx::pdl_wait();
-      for (int ks = 0; ks < pro; ++ks) {
-        ptx::mbar_arrive_expect_tx(&sh.afull[ks], C::kABytes);
-        ptx::tma_load_2d(smem + C::kOffA + ks * C::kABytes, &tm_x, &sh.afull[ks], ks * BK, m0);
-      }
-      issued_a = pro;
-      for (int ks = pro; ks < num_k; ++ks) {
-        const int s = ks % kStages;
-        const uint32_t ph = (ks / kStages) & 1;
-        if (!ptx::mbar_wait_bounded(&sh.empty[s], ph ^ 1, wait_limit, abort)) {
-          record_timeout(abort);
-          break;
+      int it = 0, tc = 0;
+      bool waited = false, ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++tc) {
+        const int tile = u / splits, sp = u % splits;
+        const int mb = tile % num_m, nb = tile / num_m;
+        const int ks0 = sp * kps, ks1 = min(num_k, ks0 + kps);
+        if (sc_tma) {
+          const int sb = tc % sc_bufs, sr = tc / sc_bufs;
+          if (sr > 0 && !ptx::mbar_wait_bounded(&sh.sempty[sb], (sr - 1) & 1, wait_limit, abort)) {
+            record_timeout(abort);
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&sh.sfull[sb], static_cast<uint32_t>(BN * (K >> 5) * 2));
+          ptx::tma_load_2d(smem + L.sc + sb * sc_bytes, &tm_s, &sh.sfull[sb], 0, nb * BN);
+          issued_s = tc + 1;
         }
-        ptx::mbar_arrive_expect_tx(&sh.wfull[s], C::kRawBytes);
-        ptx::tma_load_2d(smem + C::kOffRaw + s * C::kRawBytes, &tm_w, &sh.wfull[s],
-                         ks * C::kRawRow, n0);
-        issued_w = ks + 1;
-        ptx::mbar_arrive_expect_tx(&sh.afull[s], C::kABytes);
-        ptx::tma_load_2d(smem + C::kOffA + s * C::kABytes, &tm_x, &sh.afull[s], ks * BK, m0);
-        issued_a = ks + 1;
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
+          const int s = it % SL, r = it / SL;
+          if (r > 0 && !ptx::mbar_wait_bounded(&sh.lempty[s], (r - 1) & 1, wait_limit, abort)) {
+            record_timeout(abort);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&sh.wfull[s], kRawBytes);
+          ptx::tma_load_2d(smem + L.raw + s * kRawBytes, &tm_w, &sh.wfull[s], ks * kRawRow, nb * BN);
+          issued_w = it + 1;
+          if (!waited) {
+            ptx::pdl_wait();
+            waited = true;
+          }
+          ptx::mbar_arrive_expect_tx(&sh.afull[s], kABytes);
+          ptx::tma_load_2d(smem + L.a + s * kABytes, &tm_x, &sh.afull[s], ks * BK, mb * BM);
+          issued_a = it + 1;
+        }
       }
     }
   } else if (warp == 1) {
+    // ---- MMA issuer (one lane) ----
     if (lane == 0) {
       bool ok = true;
       // Test hook: a wait on a barrier nothing arrives on, which must run out.
@@ -233,122 +264,154 @@ __global__ void __launch_bounds__(kThreads, 1)
         record_timeout(abort);
         ok = false;
       }
-      for (int ks = 0; ks < num_k && ok; ++ks) {
-        const int s = ks % kStages;
-        const uint32_t ph = (ks / kStages) & 1;
-        ok = ptx::mbar_wait_bounded(&sh.afull[s], ph, wait_limit, abort) &&
-             ptx::mbar_wait_bounded(&sh.bfull[s], ph, wait_limit, abort);
-        if (!ok) {
+      int it = 0, tc = 0;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++tc) {
+        const int ks0 = (u % splits) * kps, ks1 = min(num_k, ks0 + kps);
+        const int ab = tc & 1, ar = tc >> 1;
+        if (ar > 0 && !ptx::mbar_wait_bounded(&sh.accempty[ab], (ar - 1) & 1, wait_limit, abort)) {
           record_timeout(abort);
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t a0 = ptx::smem_u32(smem + C::kOffA + s * C::kABytes);
-        const uint32_t b0 = ptx::smem_u32(smem + C::kOffB + s * C::kBBytes);
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          ptx::tc_mma_f16(tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), C::kIdesc,
-                          (ks | kk) != 0 ? 1u : 0u);
-        }
-        mma_issued = true;
-        ptx::tc_commit(&sh.empty[s]);
-      }
-      ptx::tc_commit(&sh.acc_full);  // also covers a partial tile after an abort
-    }
-  } else {
-    // ---- dequantisers ----
-    const int t = threadIdx.x - 64;  // 0 .. 255
-    const int spr = K >> 5;
-    constexpr int kJobs = BN * 2 / (kDequantWarps * 32);  // (row, half) jobs per thread
-    int wst0 = -kWinStages;                                // first stage of the loaded window
-    bool ok = true;
-    // Wait outcomes are made warp-uniform: the loop below contains warp-collective steps.
-    if (scales_tma &&
-        !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.sfull, 0, wait_limit, abort))) {
-      record_timeout(abort);
-      ok = false;
-    }
-    for (int ks = 0; ks < num_k && ok; ++ks) {
-      const int s = ks % kStages;
-      const uint32_t ph = (ks / kStages) & 1;
-      if (!scales_tma && ks >= wst0 + kWinStages) {
-        // This thread's own scales for the next kWinStages stages, into its private slots
-        // of shared memory (only it reads them, so no barrier is involved). Rows past N and
-        // blocks past K/32 read as zero.
-        wst0 = ks;
-#pragma unroll 4
-        for (int j = 0; j < kWinStages; ++j) {
-#pragma unroll
-          for (int jj = 0; jj < kJobs; ++jj) {
-            const int job = t + jj * kDequantWarps * 32;
-            const int gr = n0 + job % BN, kb = 2 * (ks + j) + job / BN;
-            ssc[(j * kJobs + jj) * (kDequantWarps * 32) + t] =
-                (gr < N && kb < spr) ? __ldg(scales + static_cast<size_t>(gr) * spr + kb) : 0;
+        const uint32_t d = tmem + static_cast<uint32_t>(ab * BN);
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
+          const int s = it % SL, bs = it % kSB;
+          ok = ptx::mbar_wait_bounded(&sh.afull[s], (it / SL) & 1, wait_limit, abort) &&
+               ptx::mbar_wait_bounded(&sh.bfull[bs], (it / kSB) & 1, wait_limit, abort);
+          if (!ok) {
+            record_timeout(abort);
+            break;
           }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(smem + L.a + s * kABytes);
+          const uint32_t b0 = ptx::smem_u32(smem + L.b + bs * kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            ptx::tc_mma_f16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
+                            (ks != ks0 || kk != 0) ? 1u : 0u);
+          mma_issued = true;
+          ptx::tc_commit(&sh.lempty[s]);
+          ptx::tc_commit(&sh.bempty[bs]);
         }
+        if (ok) ptx::tc_commit(&sh.accfull[ab]);
       }
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.wfull[s], ph, wait_limit, abort))) {
+      ptx::tc_commit(&sh.drain);  // arrives once every MMA issued above has completed
+    }
+  } else if (warp < 2 + kDequantWarps) {
+    // ---- dequantisers: 512 threads, one job of E codes per stage each: row t % BN, part
+    //      t / BN of the stage's 64 codes (E = 32 at BN = 256, 16 at BN = 128) ----
+    constexpr int E = BN * BK / kDequantThreads;  // codes per job
+    constexpr int CH = E / 8;                     // 16-byte B chunks per job
+    const int t = threadIdx.x - 64;
+    const int row = t % BN, part = t / BN;
+    const int spr = K >> 5;
+    const int sw = row & 7;
+    const int kbo = (part * E) >> 5;  // which 32-code block of the stage
+    int it = 0, tc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++tc) {
+      const int tile = u / splits;
+      const int ks0 = (u % splits) * kps, ks1 = min(num_k, ks0 + kps);
+      const int nb = tile / num_m;
+      const int gr = nb * BN + row;
+      const int sb = tc % sc_bufs;
+      // Wait outcomes are made warp-uniform: warp-collective steps follow.
+      if (sc_tma && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.sfull[sb], (tc / sc_bufs) & 1,
+                                                                      wait_limit, abort))) {
         record_timeout(abort);
         ok = false;
         break;
       }
-      const uint8_t *raw = smem + C::kOffRaw + s * C::kRawBytes;
-      uint8_t *btile = smem + C::kOffB + s * C::kBBytes;
-#pragma unroll
-      for (int j = 0; j < kJobs; ++j) {
-        const int job = t + j * kDequantWarps * 32;
-        const int row = job % BN, h = job / BN;  // h: which 32-element half of the stage
-        const float s0 = __half2float(__ushort_as_half(
-            scales_tma ? ssc[row * spr + 2 * ks + h]
-                       : ssc[((ks - wst0) * kJobs + j) * (kDequantWarps * 32) + t]));
-        uint8_t *brow = btile + row * 128;
-        const int sw = row & 7;
+      const uint16_t *sct = reinterpret_cast<const uint16_t *>(smem + L.sc + sb * sc_bytes);
+      for (int ks = ks0; ks < ks1; ++ks, ++it) {
+        const int s = it % SL, bs = it % kSB;
+        const int kb = 2 * ks + kbo;
+        float s0 = 0.f;
+        if (!sc_tma && gr < N && kb < spr)  // fallback: this thread's own scale from global
+          s0 = __half2float(__ushort_as_half(__ldg(scales + static_cast<size_t>(gr) * spr + kb)));
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.wfull[s], (it / SL) & 1, wait_limit, abort) &&
+                                         ptx::mbar_wait_bounded(&sh.bempty[bs], ((it / kSB) & 1) ^ 1,
+                                                                wait_limit, abort))) {
+          record_timeout(abort);
+          ok = false;
+          break;
+        }
+        if (sc_tma) s0 = __half2float(__ushort_as_half(sct[row * spr + kb]));
+        const uint8_t *raw = smem + L.raw + s * kRawBytes + row * kRawRow + part * (E * BITS / 8);
+        uint8_t *brow = smem + L.b + bs * kBBytes + row * 128;
         if constexpr (BITS == 4) {
-          const uint4 wq = *reinterpret_cast<const uint4 *>(raw + row * C::kRawRow + h * 16);
+          uint32_t ws[CH];  // one word = 8 codes = one 16-byte chunk of bf16
+          if constexpr (CH == 4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(raw);
+            ws[0] = v.x; ws[1] = v.y; ws[2] = v.z; ws[3] = v.w;
+          } else {
+            const uint2 v = *reinterpret_cast<const uint2 *>(raw);
+            ws[0] = v.x; ws[1] = v.y;
+          }
           const float sj[4] = {s0, s0 * 0.0625f, s0 * 0.00390625f, s0 * 0.000244140625f};
-          const uint32_t ws[4] = {wq.x, wq.y, wq.z, wq.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int chunk = h * 4 + i;  // 16-byte chunk = 8 bf16 = 8 elements
+          for (int i = 0; i < CH; ++i) {
+            const int chunk = part * CH + i;
             *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) = dequant_int4_word(ws[i], sj);
           }
         } else {
-          const uint4 wa = *reinterpret_cast<const uint4 *>(raw + row * C::kRawRow + h * 32);
-          const uint4 wb = *reinterpret_cast<const uint4 *>(raw + row * C::kRawRow + h * 32 + 16);
-          const uint32_t ws[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+          uint32_t ws[2 * CH];  // two words = 8 codes = one chunk
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int chunk = h * 4 + i;
+          for (int i = 0; i < CH / 2; ++i) {
+            const uint4 v = reinterpret_cast<const uint4 *>(raw)[i];
+            ws[4 * i] = v.x; ws[4 * i + 1] = v.y; ws[4 * i + 2] = v.z; ws[4 * i + 3] = v.w;
+          }
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int chunk = part * CH + i;
             *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) =
                 dequant_int8_words(ws[2 * i], ws[2 * i + 1], s0);
           }
         }
+        // Each lane makes its writes visible to the async proxy (the tensor core), the warp
+        // converges, and one lane arrives for the warp.
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&sh.bfull[bs]);
+          ptx::mbar_arrive(&sh.lempty[s]);
+        }
       }
-      // Each lane makes its tile writes visible to the async proxy (the tensor core), the
-      // warp converges, and one lane arrives for the warp.
-      ptx::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.bfull[s]);
+      if (ok && sc_tma) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.sempty[sb]);
+      }
     }
-
-    // ---- epilogue: TMEM -> registers -> Y ----
-    // Y may be read by a preceding kernel: write it only after that grid completed.
-    ptx::pdl_wait();
-    // tcgen05.ld is warp-collective, so the whole warp decides together.
-    const bool mine = ok && ptx::mbar_wait_bounded(&sh.acc_full, 0, wait_limit, abort) && !*abort;
-    const bool go = __all_sync(0xffffffffu, mine);
-    if (go) {
+  } else {
+    // ---- epilogue: TMEM accumulator -> registers -> Y ----
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const bool vec = (N & 3) == 0;
+    bool waited = false;
+    int tc = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
+      const int tile = u / splits, sp = u % splits;
+      const int mb = tile % num_m, nb = tile / num_m;
+      // One split writes Y; several write FP32 partials [split][M][N] for the reduction.
+      float *out = splits == 1 ? Y : partials + static_cast<size_t>(sp) * M * N;
+      const int ab = tc & 1;
+      if (!__all_sync(0xffffffffu,
+                      ptx::mbar_wait_bounded(&sh.accfull[ab], (tc >> 1) & 1, wait_limit, abort))) {
+        record_timeout(abort);
+        break;
+      }
       ptx::tc_fence_after();
-      const int q = warp & 3;                        // TMEM lanes 32q .. 32q+31
-      const int half = (warp - 2) >> 2;              // which half of the columns
-      const int row = m0 + q * 32 + lane;
-      const bool vec = (N & 3) == 0;
-      for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 16) {
+      if (!waited) {  // Y may be read by a preceding kernel: write it only after that grid
+        ptx::pdl_wait();
+        waited = true;
+      }
+      const int grow = mb * BM + q * 32 + lane;
+      const int n0 = nb * BN;
+      for (int c0 = 0; c0 < BN; c0 += 16) {
         uint32_t r[16];
-        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, r);
+        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * BN + c0, r);
         ptx::tmem_ld_wait();
-        if (row < M) {
-          float *yr = Y + static_cast<size_t>(row) * N + n0 + c0;
+        if (grow < M) {
+          float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
           if (vec && n0 + c0 + 16 <= N) {
 #pragma unroll
             for (int v = 0; v < 4; ++v)
@@ -362,8 +425,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-    } else if (ok && !mine) {
-      record_timeout(abort);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.accempty[ab]);
     }
   }
 
@@ -371,24 +435,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- teardown: drain what this CTA issued, then free TMEM ----
   if (warp == 0 && lane == 0 && *abort) {
-    // Only the last issue to each stage can still be in flight.
-    int no_abort = 0;
-    for (int ks = issued_w - 1; ks >= 0 && ks >= issued_w - kStages; --ks)
-      ptx::mbar_wait_bounded(&sh.wfull[ks % kStages], (ks / kStages) & 1, kDrainLimit, &no_abort);
-    for (int ks = issued_a - 1; ks >= 0 && ks >= issued_a - kStages; --ks)
-      ptx::mbar_wait_bounded(&sh.afull[ks % kStages], (ks / kStages) & 1, kDrainLimit, &no_abort);
-    if (scales_tma) ptx::mbar_wait_bounded(&sh.sfull, 0, kDrainLimit, &no_abort);
+    int no_abort = 0;  // only the last issue to each stage can still be in flight
+    for (int i = issued_w - 1; i >= 0 && i >= issued_w - SL; --i)
+      ptx::mbar_wait_bounded(&sh.wfull[i % SL], (i / SL) & 1, kDrainLimit, &no_abort);
+    for (int i = issued_a - 1; i >= 0 && i >= issued_a - SL; --i)
+      ptx::mbar_wait_bounded(&sh.afull[i % SL], (i / SL) & 1, kDrainLimit, &no_abort);
+    for (int i = issued_s - 1; i >= 0 && i >= issued_s - sc_bufs; --i)
+      ptx::mbar_wait_bounded(&sh.sfull[i % sc_bufs], (i / sc_bufs) & 1, kDrainLimit, &no_abort);
   }
-  if (warp == 1 && lane == 0 && *abort && mma_issued) {
-    // acc_full was committed after the last MMA this thread issued.
+  if (warp == 1 && lane == 0 && mma_issued) {
     int no_abort = 0;
-    ptx::mbar_wait_bounded(&sh.acc_full, 0, kDrainLimit, &no_abort);
+    ptx::mbar_wait_bounded(&sh.drain, 0, kDrainLimit, &no_abort);
   }
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, C::kTmemCols);
+    ptx::tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -407,6 +470,26 @@ __global__ void __launch_bounds__(256) x_to_bf16_kernel(const float4 *__restrict
     t = __floats2bfloat162_rn(b.x, b.y); o.z = *reinterpret_cast<uint32_t *>(&t);
     t = __floats2bfloat162_rn(b.z, b.w); o.w = *reinterpret_cast<uint32_t *>(&t);
     xb[i] = o;
+  }
+}
+
+// Y = sum over splits of the FP32 partials, in split order (deterministic); 4 per thread.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4 *__restrict__ part,
+                                                            float4 *__restrict__ y, size_t n4,
+                                                            int splits) {
+  ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float4 a = part[i];
+    for (int s = 1; s < splits; ++s) {
+      const float4 b = part[static_cast<size_t>(s) * n4 + i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    y[i] = a;
   }
 }
 
@@ -448,35 +531,46 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType type, size_t esize, const void
 
 template <int BITS, int BN>
 int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
-              cudaStream_t s, const DevInfo &dev) {
-  using C = Cfg<BITS, BN>;
-  (void)dev;
+              const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
   auto kern = qgemm_tc_kernel<BITS, BN>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
   });
   if (attr_err != cudaSuccess) return WOQ_ECUDA;
 
-  CUtensorMap tm_x, tm_w, tm_s;
+  // The whole scale tile [BN, K/32] of an output tile comes by TMA when its rows are 16-byte
+  // multiples and it is small; otherwise each dequantiser loads its own scales. Two scale
+  // buffers (the next tile's loads overlap the current tile) when shared memory still
+  // leaves at least four load stages, else one.
   const int64_t spr = w.k / 32;
-  // The whole scale tile [BN, K/32] comes by TMA when its rows are 16-byte multiples and
-  // it fits the shared-memory slot; otherwise each dequantiser loads its own scales.
-  const int scales_tma = (spr % 8 == 0 && spr <= kTmaScaleCols) ? 1 : 0;
-  if (scales_tma) {
+  const bool sc_tma = spr % 8 == 0 && spr <= kTmaScaleCols;
+  const int sc_bytes = sc_tma ? static_cast<int>((BN * spr * 2 + 127) & ~int64_t(127)) : 0;
+  const int stage = kABytes + BN * BK * BITS / 8;
+  auto stages_for = [&](int bufs) {
+    return std::min(kMaxSL, (kSmemMax - make_layout(BITS, BN, 0, sc_bytes, bufs).total) / stage);
+  };
+  int sc_bufs = sc_tma ? 2 : 1;
+  if (sc_tma && stages_for(2) < 4) sc_bufs = 1;
+  const int sl = stages_for(sc_bufs);
+  if (sl < 2) return WOQ_ESHAPE;
+  const int smem = make_layout(BITS, BN, sl, sc_bytes, sc_bufs).total;
+
+  CUtensorMap tm_x, tm_w, tm_s;
+  if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, BM,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return WOQ_ECUDA;
+  if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
+                BK * BITS / 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return WOQ_ECUDA;
+  if (sc_tma) {
     if (!make_map(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w.scales, spr, w.n,
                   static_cast<uint32_t>(spr), BN, CU_TENSOR_MAP_SWIZZLE_NONE))
       return WOQ_ECUDA;
   } else {
     std::memset(&tm_s, 0, sizeof(tm_s));
   }
-  if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, BM,
-                CU_TENSOR_MAP_SWIZZLE_128B))
-    return WOQ_ECUDA;
-  if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
-                C::kRawRow, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return WOQ_ECUDA;
 
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -498,21 +592,38 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
       return WOQ_ECUDA;
     count_launches(1);
   }
-  // 2) the GEMM.
+  // 2) the persistent GEMM: one CTA per SM (or per work unit, if fewer).
+  float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + plan.xb);
   {
+    const int64_t tiles = ((m + BM - 1) / BM) * ((w.n + BN - 1) / BN) * plan.splits;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((w.n + BN - 1) / BN),
-                       static_cast<unsigned>((m + BM - 1) / BM), 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(tiles, dev.sm_count)), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const long long lim = g_wait_limit_cycles > 0 ? g_wait_limit_cycles : kDefaultWaitLimit;
     const long long stuck = g_wait_limit_cycles < 0 ? -g_wait_limit_cycles : 0;
     if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_s, w.scales, Y, static_cast<int>(m),
-                           static_cast<int>(w.n), static_cast<int>(w.k), scales_tma, lim,
-                           stuck) != cudaSuccess)
+                           static_cast<int>(w.n), static_cast<int>(w.k), sl, sc_bytes, sc_bufs,
+                           plan.splits, partials, lim, stuck) != cudaSuccess)
+      return WOQ_ECUDA;
+    count_launches(1);
+  }
+  // 3) several K-splits: sum their partials into Y.
+  if (plan.splits > 1) {
+    const size_t n4 = static_cast<size_t>(m) * w.n / 4;
+    cudaLaunchConfig_t cfg = {};
+    size_t blocks = (n4 + 255) / 256;
+    if (blocks > static_cast<size_t>(dev.sm_count) * 8) blocks = static_cast<size_t>(dev.sm_count) * 8;
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, reinterpret_cast<const float4 *>(partials),
+                           reinterpret_cast<float4 *>(Y), n4, plan.splits) != cudaSuccess)
       return WOQ_ECUDA;
     count_launches(1);
   }
@@ -521,15 +632,37 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
 
 }  // namespace
 
-size_t gemm_tc_workspace_bytes(int64_t m, int64_t k) {
-  const size_t b = static_cast<size_t>(m) * static_cast<size_t>(k) * 2;
-  return (b + 255) & ~static_cast<size_t>(255);
+GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget) {
+  auto align = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };
+  GemmPlan p;
+  p.xb = align(static_cast<size_t>(m) * static_cast<size_t>(k) * 2);
+  const int64_t mt = (m + BM - 1) / BM;
+  const int64_t num_k = (k + BK - 1) / BK;
+  // 128 x 256 tiles do twice the work per MMA instruction; prefer them when N allows.
+  p.bn = n >= 256 ? 256 : 128;
+  int64_t tiles = mt * ((n + p.bn - 1) / p.bn);
+  // Split K until the work units cover the SMs, keeping >= 4 K-stages per split; the splits
+  // need FP32 partials in the workspace and a vectorisable Y (n % 4 == 0).
+  p.splits = 1;
+  if (n % 4 == 0 && sm_count > 0) {
+    while (p.splits < 8 && tiles * p.splits * 2 <= sm_count + sm_count / 4 &&
+           num_k / (p.splits * 2) >= 4 &&
+           p.xb + align(static_cast<size_t>(p.splits) * 2 * m * n * 4) <= budget)
+      p.splits *= 2;
+  }
+  if (p.splits == 1 && p.bn == 256 && tiles * 2 <= sm_count) p.bn = 128;  // more tiles instead
+  p.part = p.splits > 1 ? align(static_cast<size_t>(p.splits) * m * n * 4) : 0;
+  p.total = p.xb + p.part;
+  return p;
 }
 
 int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
-                   cudaStream_t s, const DevInfo &dev) {
-  return w.bits == 4 ? launch_tc<4, 128>(X, m, w, Y, workspace, s, dev)
-                     : launch_tc<8, 128>(X, m, w, Y, workspace, s, dev);
+                   const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
+  if (w.bits == 4)
+    return plan.bn == 256 ? launch_tc<4, 256>(X, m, w, Y, workspace, plan, s, dev)
+                          : launch_tc<4, 128>(X, m, w, Y, workspace, plan, s, dev);
+  return plan.bn == 256 ? launch_tc<8, 256>(X, m, w, Y, workspace, plan, s, dev)
+                        : launch_tc<8, 128>(X, m, w, Y, workspace, plan, s, dev);
 }
 
 int read_wait_timeout_flag(int clear, unsigned *value) {

@@ -34,11 +34,19 @@ int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, c
 int read_gemv_timeout_flag(int clear, unsigned *value);
 
 // ---- qgemm_tc.cu ----
-// Workspace bytes of the tensor-core path (the bf16 copy of X).
-size_t gemm_tc_workspace_bytes(int64_t m, int64_t k);
+// How the tensor-core path runs a problem: tile width, K-splits and workspace layout
+// ([bf16 copy of X][FP32 partials of the splits], each 256-byte aligned).
+struct GemmPlan {
+  int bn = 128;
+  int splits = 1;
+  size_t xb = 0, part = 0, total = 0;
+};
+// Plan for (m, n, k) on a device with sm_count SMs, using at most `budget` workspace bytes
+// (the bf16 copy of X itself is always needed).
+GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget);
 // tcgen05 bf16 GEMM: Y = bf16(X) . bf16(W_hat)^T, FP32 accumulation in tensor memory.
 int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
-                   cudaStream_t s, const DevInfo &dev);
+                   const GemmPlan &plan, cudaStream_t s, const DevInfo &dev);
 // Reads (and optionally clears) the device-side record of bounded waits that gave up on
 // the current device. Synchronous.
 int read_wait_timeout_flag(int clear, unsigned *value);
