@@ -264,9 +264,10 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
     bits = 4
     groups = UNFUSED_GROUPS if args.unfused else FUSED_GROUPS
     layers = build_decoder(bits, device, groups)
-    xs = [workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
+    M = args.m
+    xs = [workloads.activations(M, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
           for _, mem in groups]
-    ys = [torch.empty(1, group_shape(mem)[0], device=device) for _, mem in groups]
+    ys = [torch.empty(M, group_shape(mem)[0], device=device) for _, mem in groups]
     step_bytes = decode_step_bytes(layers[0])
     total_bytes = sum(decode_step_bytes(l) for l in layers)
 
@@ -290,14 +291,14 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
                 "bytes_per_launch": round(step_bytes / per_step),
                 "avg_launch_us": round(ms * 1e3 / launches, 3)}
 
-    e2e = run_decode_e2e(layers, groups, device, min(args.steps, 2000), stream, world)
+    e2e = run_decode_e2e(layers, groups, device, min(args.steps, 2000), stream, world, M)
 
     out = {
         "metric": "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)",
         "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "decoder_block_m1", "bits": 4, "block": 32, "m": 1,
+        "config": {"workload": f"decoder_block_m{M}", "bits": 4, "block": 32, "m": M,
                    "launches": [f"{nm}[{group_shape(mem)[0]}x{group_shape(mem)[1]}]"
                                 for nm, mem in groups],
                    "fused_qkv_gate_up": not args.unfused,
@@ -315,13 +316,13 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
     return out, layers, groups, xs
 
 
-def run_decode_e2e(layers, groups, device, steps, stream, world):
+def run_decode_e2e(layers, groups, device, steps, stream, world, M=1):
     """Same steps through the public API, x from pinned host memory, y read back each step."""
     import weight_only_bit_qgemv_b200 as woq
 
-    host_x = [workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).pin_memory()
+    host_x = [workloads.activations(M, group_shape(mem)[1], seed=group_x_seed(mem)).pin_memory()
               for _, mem in groups]
-    host_y = [torch.empty(1, group_shape(mem)[0]).pin_memory() for _, mem in groups]
+    host_y = [torch.empty(M, group_shape(mem)[0]).pin_memory() for _, mem in groups]
     dx = [torch.empty_like(h, device=device) for h in host_x]
     dy = [torch.empty_like(h, device=device) for h in host_y]
     h2d = sum(t.numel() * 4 for t in host_x)
@@ -540,6 +541,7 @@ def main(argv=None):
     ap.add_argument("--prefill-m", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--unfused", action="store_true", help="7 launches per block instead of 4")
+    ap.add_argument("--m", type=int, default=1, help="activation rows per decode step (1..64)")
     ap.add_argument("--no-lm-head", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -563,7 +565,7 @@ def main(argv=None):
     if not args.no_prefill:
         out["prefill"] = run_prefill(layers, groups, device, args.prefill_m, 3, peaks, peak_kind,
                                      world)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and args.m == 1:
         cb, parity = cpu_baseline_leg(layers[0], groups, xs, args.cpu_budget)
         out["cpu_baseline"] = cb
         out["parity"] = parity

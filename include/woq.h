@@ -97,9 +97,11 @@ int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, u
 
 /*
  * qgemv -- decode path, y[m, n] = x[m, k] . W_hat^T for 1 <= m <= 64 ("TinyMOSS-Diarize",
- * "How we built it": the separate GEMV path for decode). FP32 products and accumulation
- * (CUDA cores); within a 32-block the codes are multiplied exactly and the block sum is
- * scaled once. Deterministic: the same inputs give the same bits on every call.
+ * "How we built it": the separate GEMV path for decode). FP32 accuracy: within a 32-block
+ * the codes are multiplied exactly and the block sum is scaled once, in FP32. Small batches
+ * (m >= 8) over wide matrices (n / 128 >= SM count) take the tensor-core form of qgemv_path
+ * WOQ_GEMV_SPLIT_TC, every other call the CUDA-core form. Deterministic: the same inputs give
+ * the same bits on every call.
  *   x  device, [m, k] float32 row-major, 16-byte aligned
  *   w  host pointer to the weight descriptor (read during the call only)
  *   y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
@@ -107,6 +109,24 @@ int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, u
  * WOQ_ESHAPE, WOQ_EALIGN, WOQ_EDEVICE, WOQ_ECUDA.
  */
 int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream);
+
+/*
+ * qgemv_path -- qgemv with the kernel named instead of chosen by shape.
+ *   WOQ_GEMV_AUTO       as qgemv
+ *   WOQ_GEMV_CUDA_CORE  FP32 products and FP32 accumulation on the CUDA cores
+ *   WOQ_GEMV_SPLIT_TC   tensor cores: each x value is split into bf16 hi + bf16 lo
+ *                       (x - hi, rounded), the codes (exact in bf16) are multiplied against
+ *                       both in bf16 x bf16 -> FP32 MMAs, and each 32-block's FP32 sum is
+ *                       scaled by its binary16 scale in FP32. The split keeps 16 of x's 24
+ *                       significand bits; error stays within the FP32 tolerance of qgemv.
+ *                       Needs 2 <= m <= 64, k % 256 == 0 and k <= 8192, else WOQ_ESHAPE.
+ * Arguments and errors otherwise as qgemv; an unknown path is WOQ_EINVAL.
+ */
+#define WOQ_GEMV_AUTO       0
+#define WOQ_GEMV_CUDA_CORE  1
+#define WOQ_GEMV_SPLIT_TC   2
+int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t path,
+               void *stream);
 
 /*
  * Bytes of device workspace qgemm needs for (m, w, path); 0 if none. Returns 0 for

@@ -133,3 +133,72 @@ def test_launches_are_counted_and_stream_ordered():
     st.synchronize()
     assert woq.launch_count() - before == 1
     assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, 8)) <= FP32_TOL
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("m", [8, 64])
+@pytest.mark.parametrize("proj", [0, 3, 6])
+def test_small_batch_tensor_core_decoder_shapes(bits, m, proj):
+    """The tensor-core form (hi/lo bf16 split of x) keeps the FP32 tolerance."""
+    name, n, k = workloads.DECODER_PROJ[proj]
+    W = workloads.weight(n, k, seed=workloads.layer_seed(4, proj))
+    w, p, s = packed_from_weight(W, bits)
+    x = workloads.activations(m, k, seed=m)
+    buf, y = guarded_out(m, n)
+    woq.qgemv(x.cuda(), w, out=y, path="split_tc")
+    assert tail_intact(buf, m, n)
+    assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL, name
+
+
+def test_small_batch_lm_head_sampled():
+    n, k = workloads.LM_HEAD
+    W = workloads.weight(n, k, seed=workloads.LM_HEAD_SEED)
+    w, p, s = packed_from_weight(W, 8)
+    x = workloads.activations(16, k, seed=workloads.X_SEED)
+    y = woq.qgemv(x.cuda(), w).cpu().numpy()
+    rows = np.concatenate([np.random.default_rng(3).choice(n, 1024, replace=False), [n - 1]])
+    assert max_rel(y[:, rows], ref_rows(x.numpy(), p, s, 8, rows)) <= FP32_TOL
+
+
+def test_small_batch_wide_dynamic_range():
+    """x spanning many binades: the two-term split keeps ~16 bits of each value."""
+    n, k = 512, 1024
+    w, p, s = packed_raw(n, k, 4, seed=31)
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((6, k)) * np.exp(rng.uniform(-8, 8, (6, k)))).astype(np.float32)
+    y = woq.qgemv(torch.from_numpy(x).cuda(), w, path="split_tc").cpu().numpy()
+    ref = ref_rows(x, p, s, 4)
+    for r in range(6):
+        assert max_rel(y[r:r + 1], ref[r:r + 1]) <= FP32_TOL
+
+
+@pytest.mark.parametrize("m", [2, 3, 5, 17, 33])
+def test_small_batch_tensor_core_ragged_rows(m):
+    """Row counts that are not a multiple of the MMA's 8-column tile, on a ragged N."""
+    n, k = 1000, 2048
+    w, p, s = packed_raw(n, k, 4, seed=40 + m)
+    x = workloads.activations(m, k, seed=m)
+    buf, y = guarded_out(m, n)
+    woq.qgemv(x.cuda(), w, out=y, path="split_tc")
+    assert tail_intact(buf, m, n)
+    assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, 4)) <= FP32_TOL
+
+
+def test_split_tc_rejects_shapes_outside_its_limits():
+    w, _, _ = packed_raw(256, 96, 8, seed=5)  # k % 256 != 0
+    x = workloads.activations(4, 96, seed=1).cuda()
+    with pytest.raises(woq.WoqError):
+        woq.qgemv(x, w, path="split_tc")
+    x1 = workloads.activations(1, 96, seed=1).cuda()
+    with pytest.raises(woq.WoqError):
+        woq.qgemv(x1, w, path="split_tc")  # m = 1
+
+
+def test_auto_and_cuda_core_paths_agree_bitwise_on_decoder_shapes():
+    name, n, k = workloads.DECODER_PROJ[0]
+    W = workloads.weight(n, k, seed=workloads.layer_seed(0, 0))
+    w, _, _ = packed_from_weight(W, 4)
+    x = workloads.activations(8, k, seed=2).cuda()
+    a = woq.qgemv(x, w)
+    b = woq.qgemv(x, w, path="cuda_core")
+    assert torch.equal(a, b), name

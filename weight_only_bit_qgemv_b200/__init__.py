@@ -18,7 +18,15 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import WOQ_PATH_AUTO, WOQ_PATH_BF16_TC, WOQ_PATH_FP32, WoqError  # noqa: F401
+from ._lib import (  # noqa: F401
+    WOQ_GEMV_AUTO,
+    WOQ_GEMV_CUDA_CORE,
+    WOQ_GEMV_SPLIT_TC,
+    WOQ_PATH_AUTO,
+    WOQ_PATH_BF16_TC,
+    WOQ_PATH_FP32,
+    WoqError,
+)
 
 __all__ = [
     "PackedWeight",
@@ -33,6 +41,7 @@ __all__ = [
 ]
 
 _PATHS = {"auto": WOQ_PATH_AUTO, "fp32": WOQ_PATH_FP32, "bf16_tc": WOQ_PATH_BF16_TC}
+_GEMV_PATHS = {"auto": WOQ_GEMV_AUTO, "cuda_core": WOQ_GEMV_CUDA_CORE, "split_tc": WOQ_GEMV_SPLIT_TC}
 
 
 def _ptr(t: torch.Tensor) -> int:
@@ -88,15 +97,23 @@ def pack(W: torch.Tensor, bits: int, device="cuda") -> PackedWeight:
     return PackedWeight(packed.to(device), scales.to(device), bits, n, k)
 
 
-def qgemv(x: torch.Tensor, w: PackedWeight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y[m, n] = x[m, k] . W_hat^T, 1 <= m <= 64, FP32 (C ABI ``qgemv``)."""
+def qgemv(
+    x: torch.Tensor,
+    w: PackedWeight,
+    out: torch.Tensor | None = None,
+    stream=None,
+    path: str = "auto",
+) -> torch.Tensor:
+    """y[m, n] = x[m, k] . W_hat^T, 1 <= m <= 64, FP32 accuracy (C ABI ``qgemv_path``);
+    path in {"auto", "cuda_core", "split_tc"}."""
     if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
         raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
     m = x.shape[0]
     if out is None:
         out = torch.empty(m, w.n, dtype=torch.float32, device=x.device)
     d = w.desc()
-    _lib.check(_lib.lib().qgemv(_ptr(x), m, ctypes.byref(d), _ptr(out), _stream(stream)), "qgemv")
+    rc = _lib.lib().qgemv_path(_ptr(x), m, ctypes.byref(d), _ptr(out), _GEMV_PATHS[path], _stream(stream))
+    _lib.check(rc, "qgemv")
     return out
 
 

@@ -21,11 +21,15 @@ WOQ_EWORKSPACE = -8
 WOQ_PATH_AUTO = 0
 WOQ_PATH_FP32 = 1
 WOQ_PATH_BF16_TC = 2
+WOQ_GEMV_AUTO = 0
+WOQ_GEMV_CUDA_CORE = 1
+WOQ_GEMV_SPLIT_TC = 2
 
 #: Every symbol include/woq.h declares.
 EXPORTS = (
     "qpack",
     "qgemv",
+    "qgemv_path",
     "qgemm_workspace_bytes",
     "qgemm",
     "qgemm_bf16_noalloc",
@@ -74,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.qpack.restype = ctypes.c_int
     L.qgemv.argtypes = [vp, c_i64, wp, vp, vp]
     L.qgemv.restype = ctypes.c_int
+    L.qgemv_path.argtypes = [vp, c_i64, wp, vp, c_i32, vp]
+    L.qgemv_path.restype = ctypes.c_int
     L.qgemm_workspace_bytes.argtypes = [c_i64, wp, c_i32]
     L.qgemm_workspace_bytes.restype = ctypes.c_size_t
     L.qgemm.argtypes = [vp, c_i64, wp, vp, c_i32, vp, ctypes.c_size_t, vp]

@@ -66,17 +66,37 @@ using woq::DevInfo;
 
 extern "C" {
 
-int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream) {
+// qgemv runs on the tensor cores from this many activation rows on, for matrices wide
+// enough that 128-row tiles cover every SM; measured on B200, the CUDA-core kernel is faster
+// for fewer rows and for the narrower decoder projections.
+constexpr int64_t kTcMinM = 8;
+
+int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t path,
+               void *stream) {
   int rc = woq::check_weight(w);
   if (rc != WOQ_OK) return rc;
   if (!x || !y) return WOQ_EINVAL;
   if (m < 1 || m > 64) return WOQ_EINVAL;
+  if (path != WOQ_GEMV_AUTO && path != WOQ_GEMV_CUDA_CORE && path != WOQ_GEMV_SPLIT_TC)
+    return WOQ_EINVAL;
   if (w->k > 32768) return WOQ_ESHAPE;
   if (!woq::aligned(x, 16) || !woq::aligned(y, 16)) return WOQ_EALIGN;
   DevInfo dev;
   rc = woq::current_device(&dev);
   if (rc != WOQ_OK) return rc;
-  return woq::launch_gemv_fp32(x, m, *w, y, static_cast<cudaStream_t>(stream), dev, true);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tc = path == WOQ_GEMV_SPLIT_TC ||
+                  (path == WOQ_GEMV_AUTO && m >= kTcMinM && (w->n + 127) / 128 >= dev.sm_count);
+  if (tc) {
+    rc = woq::launch_gemv_tc(x, m, *w, y, s, dev);
+    if (rc != 1) return rc;
+    if (path == WOQ_GEMV_SPLIT_TC) return WOQ_ESHAPE;  // shape outside the kernel's limits
+  }
+  return woq::launch_gemv_fp32(x, m, *w, y, s, dev, true);
+}
+
+int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream) {
+  return qgemv_path(x, m, w, y, WOQ_GEMV_AUTO, stream);
 }
 
 // SM count the tensor-core plan is made for: the current device's, or 0 (no K-splits) when
@@ -124,12 +144,14 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
 
 int woq_device_status(int clear) {
   if (cudaDeviceSynchronize() != cudaSuccess) return WOQ_ECUDA;
-  unsigned v = 0, g = 0;
+  unsigned v = 0, g = 0, t = 0;
   int rc = woq::read_wait_timeout_flag(clear, &v);
   if (rc != WOQ_OK) return rc;
   rc = woq::read_gemv_timeout_flag(clear, &g);
   if (rc != WOQ_OK) return rc;
-  return (v || g) ? WOQ_ETIMEOUT : WOQ_OK;
+  rc = woq::read_gemv_tc_timeout_flag(clear, &t);
+  if (rc != WOQ_OK) return rc;
+  return (v || g || t) ? WOQ_ETIMEOUT : WOQ_OK;
 }
 
 void woq_debug_set_wait_limit(long long cycles) { woq::set_wait_limit_cycles(cycles); }

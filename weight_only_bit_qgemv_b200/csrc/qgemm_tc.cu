@@ -213,50 +213,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  int issued_w = 0, issued_a = 0, issued_s = 0;  // producer bookkeeping for the drain
+  // producer bookkeeping for the drain: slots issued at least once, and the parity of
+  // their last issue
+  uint32_t wmask = 0, wpar = 0, amask = 0, apar = 0, smask = 0, spar = 0;
   bool mma_issued = false;
 
   if (warp == 0) {
     // ---- producer (one lane). Only X depends on preceding kernels: wait before it. ----
+    // Ring positions advance incrementally (no division on the issue path); a wait with the
+    // opposite parity passes at once on a fresh barrier, so the first round needs no case.
     if (lane == 0) {
-      int it = 0, tc = 0;
+      int s = 0, sb = 0;
+      uint32_t ph = 0, sph = 0;
       bool waited = false, ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++tc) {
-        const int tile = u / splits, sp = u % splits;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const int tile = u / splits, sp = u - (u / splits) * splits;
         const int mb = tile % num_m, nb = tile / num_m;
         const int ks0 = sp * kps, ks1 = min(num_k, ks0 + kps);
         if (sc_tma) {
-          const int sb = tc % sc_bufs, sr = tc / sc_bufs;
-          if (sr > 0 && !ptx::mbar_wait_bounded(&sh.sempty[sb], (sr - 1) & 1, wait_limit, abort)) {
+          if (!ptx::mbar_wait_bounded(&sh.sempty[sb], sph ^ 1, wait_limit, abort)) {
             record_timeout(abort);
             break;
           }
           ptx::mbar_arrive_expect_tx(&sh.sfull[sb], static_cast<uint32_t>(BN * (K >> 5) * 2));
           ptx::tma_load_2d(smem + L.sc + sb * sc_bytes, &tm_s, &sh.sfull[sb], 0, nb * BN);
-          issued_s = tc + 1;
+          smask |= 1u << sb;
+          spar = (spar & ~(1u << sb)) | (sph << sb);
+          if (++sb == sc_bufs) {
+            sb = 0;
+            sph ^= 1;
+          }
         }
-        for (int ks = ks0; ks < ks1; ++ks, ++it) {
-          const int s = it % SL, r = it / SL;
-          if (r > 0 && !ptx::mbar_wait_bounded(&sh.lempty[s], (r - 1) & 1, wait_limit, abort)) {
+        for (int ks = ks0; ks < ks1; ++ks) {
+          if (!ptx::mbar_wait_bounded(&sh.lempty[s], ph ^ 1, wait_limit, abort)) {
             record_timeout(abort);
             ok = false;
             break;
           }
           ptx::mbar_arrive_expect_tx(&sh.wfull[s], kRawBytes);
           ptx::tma_load_2d(smem + L.raw + s * kRawBytes, &tm_w, &sh.wfull[s], ks * kRawRow, nb * BN);
-          issued_w = it + 1;
+          wmask |= 1u << s;
+          wpar = (wpar & ~(1u << s)) | (ph << s);
           if (!waited) {
             ptx::pdl_wait();
             waited = true;
           }
           ptx::mbar_arrive_expect_tx(&sh.afull[s], kABytes);
           ptx::tma_load_2d(smem + L.a + s * kABytes, &tm_x, &sh.afull[s], ks * BK, mb * BM);
-          issued_a = it + 1;
+          amask |= 1u << s;
+          apar = (apar & ~(1u << s)) | (ph << s);
+          if (++s == SL) {
+            s = 0;
+            ph ^= 1;
+          }
         }
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer (one lane) ----
+    // ---- MMA issuer (one lane): descriptors advance by constants, no division ----
     if (lane == 0) {
       bool ok = true;
       // Test hook: a wait on a barrier nothing arrives on, which must run out.
@@ -264,36 +278,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         record_timeout(abort);
         ok = false;
       }
-      int it = 0, tc = 0;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++tc) {
-        const int ks0 = (u % splits) * kps, ks1 = min(num_k, ks0 + kps);
-        const int ab = tc & 1, ar = tc >> 1;
-        if (ar > 0 && !ptx::mbar_wait_bounded(&sh.accempty[ab], (ar - 1) & 1, wait_limit, abort)) {
+      const uint64_t adesc0 = sw128_desc(ptx::smem_u32(smem + L.a));
+      const uint64_t bdesc0 = sw128_desc(ptx::smem_u32(smem + L.b));
+      int s = 0, bs = 0, ab = 0;
+      uint32_t ph = 0, bph = 0, aph = 0;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const int ks0 = (u - (u / splits) * splits) * kps, ks1 = min(num_k, ks0 + kps);
+        if (!ptx::mbar_wait_bounded(&sh.accempty[ab], aph ^ 1, wait_limit, abort)) {
           record_timeout(abort);
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(ab * BN);
-        for (int ks = ks0; ks < ks1; ++ks, ++it) {
-          const int s = it % SL, bs = it % kSB;
-          ok = ptx::mbar_wait_bounded(&sh.afull[s], (it / SL) & 1, wait_limit, abort) &&
-               ptx::mbar_wait_bounded(&sh.bfull[bs], (it / kSB) & 1, wait_limit, abort);
+        for (int ks = ks0; ks < ks1; ++ks) {
+          ok = ptx::mbar_wait_bounded(&sh.afull[s], ph, wait_limit, abort) &&
+               ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort);
           if (!ok) {
             record_timeout(abort);
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a0 = ptx::smem_u32(smem + L.a + s * kABytes);
-          const uint32_t b0 = ptx::smem_u32(smem + L.b + bs * kBBytes);
+          // start-address field counts 16-byte units; K=16 bf16 = 32 bytes = 2 units
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kABytes >> 4));
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>(bs * (kBBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            ptx::tc_mma_f16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
-                            (ks != ks0 || kk != 0) ? 1u : 0u);
+            ptx::tc_mma_f16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
           mma_issued = true;
           ptx::tc_commit(&sh.lempty[s]);
           ptx::tc_commit(&sh.bempty[bs]);
+          if (++s == SL) {
+            s = 0;
+            ph ^= 1;
+          }
+          if (++bs == kSB) {
+            bs = 0;
+            bph ^= 1;
+          }
         }
-        if (ok) ptx::tc_commit(&sh.accfull[ab]);
+        if (!ok) break;
+        ptx::tc_commit(&sh.accfull[ab]);
+        if (++ab == 2) {
+          ab = 0;
+          aph ^= 1;
+        }
       }
       ptx::tc_commit(&sh.drain);  // arrives once every MMA issued above has completed
     }
@@ -307,31 +335,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int spr = K >> 5;
     const int sw = row & 7;
     const int kbo = (part * E) >> 5;  // which 32-code block of the stage
-    int it = 0, tc = 0;
+    int s = 0, bs = 0, sb = 0;
+    uint32_t ph = 0, bph = 0, sph = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++tc) {
+    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
       const int tile = u / splits;
-      const int ks0 = (u % splits) * kps, ks1 = min(num_k, ks0 + kps);
+      const int ks0 = (u - tile * splits) * kps, ks1 = min(num_k, ks0 + kps);
       const int nb = tile / num_m;
       const int gr = nb * BN + row;
-      const int sb = tc % sc_bufs;
       // Wait outcomes are made warp-uniform: warp-collective steps follow.
-      if (sc_tma && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.sfull[sb], (tc / sc_bufs) & 1,
-                                                                      wait_limit, abort))) {
+      if (sc_tma && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.sfull[sb], sph, wait_limit, abort))) {
         record_timeout(abort);
         ok = false;
         break;
       }
       const uint16_t *sct = reinterpret_cast<const uint16_t *>(smem + L.sc + sb * sc_bytes);
-      for (int ks = ks0; ks < ks1; ++ks, ++it) {
-        const int s = it % SL, bs = it % kSB;
+      for (int ks = ks0; ks < ks1; ++ks) {
         const int kb = 2 * ks + kbo;
         float s0 = 0.f;
         if (!sc_tma && gr < N && kb < spr)  // fallback: this thread's own scale from global
           s0 = __half2float(__ushort_as_half(__ldg(scales + static_cast<size_t>(gr) * spr + kb)));
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.wfull[s], (it / SL) & 1, wait_limit, abort) &&
-                                         ptx::mbar_wait_bounded(&sh.bempty[bs], ((it / kSB) & 1) ^ 1,
-                                                                wait_limit, abort))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.wfull[s], ph, wait_limit, abort) &&
+                                         ptx::mbar_wait_bounded(&sh.bempty[bs], bph ^ 1, wait_limit, abort))) {
           record_timeout(abort);
           ok = false;
           break;
@@ -376,10 +401,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::mbar_arrive(&sh.bfull[bs]);
           ptx::mbar_arrive(&sh.lempty[s]);
         }
+        if (++s == SL) {
+          s = 0;
+          ph ^= 1;
+        }
+        if (++bs == kSB) {
+          bs = 0;
+          bph ^= 1;
+        }
       }
       if (ok && sc_tma) {
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.sempty[sb]);
+        if (++sb == sc_bufs) {
+          sb = 0;
+          sph ^= 1;
+        }
       }
     }
   } else {
@@ -387,15 +424,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
     const bool vec = (N & 3) == 0;
     bool waited = false;
-    int tc = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
-      const int tile = u / splits, sp = u % splits;
+    int ab = 0;
+    uint32_t aph = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const int tile = u / splits, sp = u - tile * splits;
       const int mb = tile % num_m, nb = tile / num_m;
       // One split writes Y; several write FP32 partials [split][M][N] for the reduction.
       float *out = splits == 1 ? Y : partials + static_cast<size_t>(sp) * M * N;
-      const int ab = tc & 1;
-      if (!__all_sync(0xffffffffu,
-                      ptx::mbar_wait_bounded(&sh.accfull[ab], (tc >> 1) & 1, wait_limit, abort))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.accfull[ab], aph, wait_limit, abort))) {
         record_timeout(abort);
         break;
       }
@@ -428,6 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&sh.accempty[ab]);
+      if (++ab == 2) {
+        ab = 0;
+        aph ^= 1;
+      }
     }
   }
 
@@ -435,13 +475,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- teardown: drain what this CTA issued, then free TMEM ----
   if (warp == 0 && lane == 0 && *abort) {
-    int no_abort = 0;  // only the last issue to each stage can still be in flight
-    for (int i = issued_w - 1; i >= 0 && i >= issued_w - SL; --i)
-      ptx::mbar_wait_bounded(&sh.wfull[i % SL], (i / SL) & 1, kDrainLimit, &no_abort);
-    for (int i = issued_a - 1; i >= 0 && i >= issued_a - SL; --i)
-      ptx::mbar_wait_bounded(&sh.afull[i % SL], (i / SL) & 1, kDrainLimit, &no_abort);
-    for (int i = issued_s - 1; i >= 0 && i >= issued_s - sc_bufs; --i)
-      ptx::mbar_wait_bounded(&sh.sfull[i % sc_bufs], (i / sc_bufs) & 1, kDrainLimit, &no_abort);
+    int no_abort = 0;  // only the last issue to each slot can still be in flight
+    for (int i = 0; i < SL; ++i) {
+      if ((wmask >> i) & 1)
+        ptx::mbar_wait_bounded(&sh.wfull[i], (wpar >> i) & 1, kDrainLimit, &no_abort);
+      if ((amask >> i) & 1)
+        ptx::mbar_wait_bounded(&sh.afull[i], (apar >> i) & 1, kDrainLimit, &no_abort);
+    }
+    for (int i = 0; i < sc_bufs; ++i)
+      if ((smask >> i) & 1)
+        ptx::mbar_wait_bounded(&sh.sfull[i], (spar >> i) & 1, kDrainLimit, &no_abort);
   }
   if (warp == 1 && lane == 0 && mma_issued) {
     int no_abort = 0;
@@ -514,21 +557,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D tensor map over a row-major [rows, cols] array.
-bool make_map(CUtensorMap *m, CUtensorMapDataType type, size_t esize, const void *base,
-              uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-              CUtensorMapSwizzle swz) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * esize};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int BITS, int BN>
 int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
               const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
@@ -558,14 +586,14 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   const int smem = make_layout(BITS, BN, sl, sc_bytes, sc_bufs).total;
 
   CUtensorMap tm_x, tm_w, tm_s;
-  if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, BM,
+  if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, BM,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return WOQ_ECUDA;
-  if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
+  if (!make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
                 BK * BITS / 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return WOQ_ECUDA;
   if (sc_tma) {
-    if (!make_map(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w.scales, spr, w.n,
+    if (!make_tensor_map_2d(&tm_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w.scales, spr, w.n,
                   static_cast<uint32_t>(spr), BN, CU_TENSOR_MAP_SWIZZLE_NONE))
       return WOQ_ECUDA;
   } else {
@@ -631,6 +659,22 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
 }
 
 }  // namespace
+
+// 2-D tensor map over a row-major [rows, cols] array.
+bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType type, size_t esize, const void *base,
+              uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+              CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * esize};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 
 GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget) {
   auto align = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };

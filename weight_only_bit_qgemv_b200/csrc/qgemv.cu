@@ -600,22 +600,29 @@ struct OccHash {
   }
 };
 
-// Resident CTAs per SM for (kernel, dynamic smem) on the device; also raises the
-// kernel's dynamic shared memory limit when needed. Cached.
-int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev, int threads = kThreads) {
+// Resident CTAs per SM for (kernel, dynamic smem) on the device. Cached. Every kernel's
+// dynamic shared-memory limit is raised once per device, on first use, to the most any of
+// its launches asks for (`smem_max`), so that no launch depends on which sizes came first.
+int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev, int threads, size_t smem_max) {
   static std::mutex mu;
   static std::unordered_map<OccKey, int, OccHash> cache;
   const OccKey key{fn, smem, dev.device};
+  const OccKey raised{fn, 0, dev.device};
+  bool need_raise = false;
   {
     std::lock_guard<std::mutex> g(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
+    need_raise = cache.find(raised) == cache.end();
   }
-  if (smem > 48 * 1024) {
+  if (need_raise) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+                             static_cast<int>(smem_max)) != cudaSuccess)
       return -1;
+    std::lock_guard<std::mutex> g(mu);
+    cache[raised] = 1;
   }
+  if (smem > smem_max) return -1;
   int nb = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem) != cudaSuccess)
     return -1;
@@ -624,12 +631,15 @@ int blocks_per_sm(const void *fn, size_t smem, const DevInfo &dev, int threads =
   return nb;
 }
 
+constexpr size_t kRegSmemMax = 200 * 1024;  // x rows staged by the register-path kernel
+
 template <int BITS, int MT, int R, int U>
 int launch_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
              const DevInfo &dev, bool pdl) {
   auto kern = gemv_kernel<BITS, MT, R, U>;
   const size_t smem = static_cast<size_t>(MT) * w.k * sizeof(float);
-  const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev);
+  const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev, kThreads,
+                               kRegSmemMax);
   if (nb <= 0) return WOQ_ECUDA;
   const int64_t units = (w.n + R - 1) / R;
   int64_t gx = (units + kWarps - 1) / kWarps;
@@ -696,7 +706,8 @@ int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cuda
                       static_cast<int64_t>(stage_bytes);
   stages = std::max<int64_t>(1, std::min<int64_t>({stages, fit, kMaxStages}));
   const size_t smem = kBulkHeader + x_bytes + stages * stage_bytes;
-  const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev, kBulkThreads);
+  const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev, kBulkThreads,
+                               kCtaSmemBudget);
   if (nb <= 0) return WOQ_ECUDA;
   const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(num_tiles, static_cast<int64_t>(dev.sm_count) * nb));
   const int64_t gy = (m + MT - 1) / MT;
@@ -744,7 +755,7 @@ template <int BITS>
 int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
             const DevInfo &dev, bool pdl) {
   int mt = m == 1 ? 1 : m == 2 ? 2 : m <= 4 ? 4 : 8;
-  const size_t limit = dev.smem_optin < 200 * 1024 ? dev.smem_optin : 200 * 1024;
+  const size_t limit = dev.smem_optin < kRegSmemMax ? dev.smem_optin : kRegSmemMax;
   while (mt > 1 && static_cast<size_t>(mt) * w.k * sizeof(float) > limit) mt /= 2;
   if (static_cast<size_t>(mt) * w.k * sizeof(float) > limit) return WOQ_ESHAPE;
   int rc = 1;

@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "woq.h"
@@ -24,6 +25,12 @@ int current_device(DevInfo *out);
 // Adds n to the process-wide launch counter reported by woq_launch_count().
 void count_launches(uint64_t n);
 
+// 2-D tensor map (TMA descriptor) over a row-major [rows, cols] array of `esize`-byte
+// elements, box [box_rows, box_cols]; false if the driver refuses it. (qgemm_tc.cu)
+bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType type, size_t esize, const void *base,
+                        uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                        CUtensorMapSwizzle swz);
+
 // ---- qgemv.cu ----
 // FP32 CUDA-core GEMV/GEMM: y[m, n] = x[m, k] . W_hat^T for any m >= 1. Arguments
 // already validated. `pdl` launches with programmatic stream serialization.
@@ -32,6 +39,13 @@ int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, c
 
 // Reads (and optionally clears) the GEMV kernels' record of bounded waits that gave up.
 int read_gemv_timeout_flag(int clear, unsigned *value);
+
+// ---- qgemv_tc.cu ----
+// Small-batch GEMV on tensor cores (2 <= m <= 64, FP32-accurate via a hi/lo bf16 split of x).
+// Returns 1 (nothing launched) for shapes it does not take.
+int launch_gemv_tc(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                   const DevInfo &dev);
+int read_gemv_tc_timeout_flag(int clear, unsigned *value);
 
 // ---- qgemm_tc.cu ----
 // How the tensor-core path runs a problem: tile width, K-splits and workspace layout
