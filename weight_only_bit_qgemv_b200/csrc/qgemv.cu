@@ -428,8 +428,12 @@ __global__ void __launch_bounds__(kThreads)
 // partial last tile is read straight from global memory by the compute warps.
 // ---------------------------------------------------------------------------------------
 
-constexpr int kBulkWarps = 8;
-constexpr int kBulkThreads = (kBulkWarps + 1) * 32;
+// Compute warps per CTA (NW): 8, or 16 for a single activation row over a matrix small
+// enough that every CTA sees at most a couple of tiles. There the launch is latency-bound:
+// the arithmetic after x arrives is on the critical path and twice the warps halve it,
+// while two such CTAs (registers capped for it) still fit on an SM, so the next launch's
+// CTAs can stream their weights beside this one's.
+__host__ __device__ constexpr int bulk_threads(int nw) { return (nw + 1) * 32; }
 constexpr int kMaxStages = 8;
 constexpr int kBulkHeader = 256;  // mbarriers + abort flag (BulkShared, padded)
 constexpr long long kGemvWaitLimit = 1LL << 32;   // cycles (~2 s)
@@ -447,11 +451,12 @@ __device__ __forceinline__ void gemv_record_timeout(volatile int *abort) {
   atomicOr(&g_gemv_timeout_flag, 1u);
 }
 
-template <int BITS, int MT, int RW>
-__global__ void __launch_bounds__(kBulkThreads)
+template <int BITS, int MT, int RW, int NW>
+__global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
                      const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n,
                      int k, int stages, int stage_bytes, int x_bytes) {
+  constexpr int kBulkWarps = NW;
   constexpr int TR = kBulkWarps * RW;
   extern __shared__ __align__(128) uint8_t smem[];
   BulkShared &sh = *reinterpret_cast<BulkShared *>(smem);
@@ -464,7 +469,6 @@ __global__ void __launch_bounds__(kBulkThreads)
   const int warp = tid >> 5;
   const int m0 = blockIdx.y * MT;
   const int units_row = k >> 2;
-  const int cpr = (k * BITS) >> 7;
   const int spr = k >> 5;
   const size_t row_bytes = static_cast<size_t>(k) * BITS / 8;
   const uint32_t code_bytes = static_cast<uint32_t>(TR * row_bytes);
@@ -692,11 +696,12 @@ int pick_ru(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
 constexpr size_t kStageTarget = 20 * 1024;   // bytes per ring stage to aim for
 constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
 
-template <int BITS, int MT, int RW>
+template <int BITS, int MT, int RW, int NW>
 int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                   const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes) {
-  auto kern = gemv_bulk_kernel<BITS, MT, RW>;
-  constexpr int TR = kBulkWarps * RW;
+  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW>;
+  constexpr int kBulkThreads = bulk_threads(NW);
+  constexpr int TR = NW * RW;
   const int64_t num_tiles = (w.n + TR - 1) / TR;
   const int64_t full_tiles = w.n / TR;
   // stages: enough for the tiles one CTA will see, within the smem budget
@@ -731,24 +736,46 @@ int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cuda
   return WOQ_OK;
 }
 
+// Rows per warp for NW compute warps: as many as fit a stage of about kStageTarget bytes.
+inline int bulk_rows_per_warp(int nw, int rw_max, size_t row_total) {
+  int rw = rw_max;
+  while (rw > 1 && static_cast<size_t>(nw) * rw * row_total > kStageTarget) rw /= 2;
+  return rw;
+}
+
+template <int BITS, int MT, int NW>
+int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                   const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes) {
+  // More rows per warp only where registers allow.
+  int rw = bulk_rows_per_warp(NW, NW == 16 ? 2 : MT <= 2 ? 4 : 2, row_total);
+  const size_t stage_bytes = (static_cast<size_t>(NW) * rw * row_total + 127) & ~size_t(127);
+  if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return 1;
+  if (w.n < NW * rw) rw = 1;  // tiny n: one row per warp, all from global memory
+  if constexpr (MT <= 2 && NW == 8) {
+    if (rw == 4) return launch_bulk_t<BITS, MT, 4, NW>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+  }
+  if constexpr (NW == 8 || MT == 1) {
+    if (rw >= 2) return launch_bulk_t<BITS, MT, 2, NW>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+  }
+  return launch_bulk_t<BITS, MT, 1, NW>(x, m, w, y, s, dev, pdl,
+                                        (static_cast<size_t>(NW) * row_total + 127) & ~size_t(127), x_bytes);
+}
+
 template <int BITS, int MT>
 int try_bulk(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
              const DevInfo &dev, bool pdl) {
   const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
   const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
-  int rw = MT <= 2 ? 4 : 2;  // more rows per warp only where registers allow
-  while (rw > 1 && kBulkWarps * rw * row_total > kStageTarget) rw /= 2;
-  const size_t stage_bytes = (kBulkWarps * rw * row_total + 127) & ~size_t(127);
-  if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return 1;
-  if (w.n < kBulkWarps * rw) rw = 1;  // tiny n: one row per warp, all from global memory
-  if constexpr (MT <= 2) {
-    if (rw == 4) return launch_bulk_t<BITS, MT, 4>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+  if constexpr (MT == 1) {
+    // 16 warps where each CTA of the grid gets at most two tiles (latency-bound launches).
+    const int rw16 = bulk_rows_per_warp(16, 2, row_total);
+    const int64_t tiles16 = w.n / (16 * rw16);
+    if (tiles16 >= 1 && tiles16 <= 2 * static_cast<int64_t>(dev.sm_count)) {
+      const int rc = launch_bulk_nw<BITS, MT, 16>(x, m, w, y, s, dev, pdl, row_total, x_bytes);
+      if (rc != 1) return rc;
+    }
   }
-  switch (rw) {
-    case 2: return launch_bulk_t<BITS, MT, 2>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
-    default: return launch_bulk_t<BITS, MT, 1>(x, m, w, y, s, dev, pdl,
-                                             (kBulkWarps * row_total + 127) & ~size_t(127), x_bytes);
-  }
+  return launch_bulk_nw<BITS, MT, 8>(x, m, w, y, s, dev, pdl, row_total, x_bytes);
 }
 
 template <int BITS>
