@@ -47,6 +47,34 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 1024 * 1024
 
 
+def measured_traffic(workload: str, root: str | None = None):
+    """DRAM bytes per launch for `workload` from profiles/traffic.txt (an ncu capture), or None
+    when there is none or a kernel source it was taken with has changed since."""
+    import hashlib
+
+    root = root or os.path.dirname(os.path.abspath(__file__))
+    path = os.path.join(root, "profiles", "traffic.txt")
+    csrc = os.path.join(root, "weight_only_bit_qgemv_b200", "csrc")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    for line in lines:
+        f = line.split()
+        if not f or f[0].startswith("#") or f[0] != workload:
+            continue
+        for dep in f[3:]:
+            name, digest = dep.split("=")
+            try:
+                now = hashlib.sha256(open(os.path.join(csrc, name), "rb").read()).hexdigest()[:16]
+            except OSError:
+                return None
+            if now != digest:
+                return None
+        return int(f[1])
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -287,7 +315,9 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
     achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "peak_source": peak_kind,
+                "traffic": (measured_traffic("decoder_block_m1")
+                            if M == 1 and not args.unfused else None),
+                "peak_source": peak_kind,
                 "bytes_per_launch": round(step_bytes / per_step),
                 "avg_launch_us": round(ms * 1e3 / launches, 3)}
 
@@ -382,6 +412,7 @@ def run_lm_head_roofline(device, peaks, peak_kind, reps=20):
     gbs = w0.nbytes / (med / 1e3) / 1e9
     return {"workload": "lm_head_m1_int8", "weight_bytes": w0.nbytes, "launch_us_median": med * 1e3,
             "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "traffic": measured_traffic("lm_head_m1_int8"),
             "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peak_kind,
             "timing": f"median of {reps} single launches, CUDA events, two alternating copies"}
 

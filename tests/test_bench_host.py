@@ -53,3 +53,32 @@ def test_single_rank_is_identity():
 
     value, ms = bench.aggregate_throughput(5e8, 2.0, 1)
     assert ms == 2.0 and value == pytest.approx(5e8 / 2e-3)
+
+
+def test_measured_traffic_goes_null_when_the_kernel_source_changes(tmp_path):
+    import hashlib
+
+    import bench
+
+    csrc = tmp_path / "weight_only_bit_qgemv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cu").write_text("kernel v1\n")
+    digest = hashlib.sha256(b"kernel v1\n").hexdigest()[:16]
+    (tmp_path / "profiles" / "traffic.txt").write_text(
+        "# comment\nwork_a 12345 summary.md k.cu=%s\nwork_b 7 summary.md\n" % digest)
+    assert bench.measured_traffic("work_a", str(tmp_path)) == 12345
+    assert bench.measured_traffic("work_b", str(tmp_path)) == 7
+    assert bench.measured_traffic("missing", str(tmp_path)) is None
+    (csrc / "k.cu").write_text("kernel v2\n")
+    assert bench.measured_traffic("work_a", str(tmp_path)) is None
+    (csrc / "k.cu").unlink()
+    assert bench.measured_traffic("work_a", str(tmp_path)) is None
+
+
+def test_committed_traffic_file_parses():
+    import bench
+
+    for workload in ("decoder_block_m1", "lm_head_m1_int8"):
+        v = bench.measured_traffic(workload)
+        assert v is None or v > 0
