@@ -4,17 +4,19 @@
 // each weight tile is dequantised once into shared memory per (output tile, K-stage) and
 // read by the tensor core for all 128 rows of the M-tile.
 //
-// Persistent, warp-specialised kernel; one CTA per SM walks 128 x 128 output tiles.
+// Persistent, warp-specialised kernel; one CTA per SM walks (128 * MH) x BN output tiles.
 //   warp 0        producer: bulk tensor copies (TMA, no multicast) of the bf16 X tile
-//                 (128B-swizzled) and the raw code tile into a ring of SL load stages, and
-//                 of each output tile's [128, K/32] scale tile into a double buffer
-//   warp 1        TMEM owner; one thread issues tcgen05.mma (M=128, N=128, K=16, bf16 x
-//                 bf16 -> f32) into one of two accumulators and commits completions
-//   warps 2..9    dequantisers: raw codes + binary16 scales -> bf16(scale * code) written
+//                 (128B-swizzled, 128 * MH rows) and the raw code tile into a ring of SL load
+//                 stages, and of each output tile's [BN, K/32] scale tile into a double buffer
+//   warp 1        TMEM owner; one thread issues tcgen05.mma (M=128, N=BN, K=16, bf16 x
+//                 bf16 -> f32), one per 128-row half of the tile, into one of two accumulator
+//                 sets and commits completions
+//   warps 2..17   dequantisers: raw codes + binary16 scales -> bf16(scale * code) written
 //                 into a short ring of B tiles in the 128B-swizzled K-major layout that the
-//                 MMA's shared-memory descriptor names
-//   warps 10..13  epilogue: tcgen05.ld of the finished accumulator -> FP32 Y, while the MMA
-//                 thread already fills the other accumulator with the next tile
+//                 MMA's shared-memory descriptor names; with MH = 2 each B tile feeds both
+//                 halves, so the dequantisation per FLOP is halved
+//   warps 18..21  epilogue: tcgen05.ld of the finished accumulators -> FP32 Y, while the MMA
+//                 thread already fills the other set with the next tile
 // Every mbarrier wait is bounded. A wait that gives up records the event in a device flag
 // and stops the CTA's other roles; the CTA drains the copies and MMAs it issued, frees
 // tensor memory and returns.
@@ -76,11 +78,12 @@ struct Shared {
 struct Layout {
   int a, b, raw, sc, bar, total;
 };
-__host__ __device__ inline Layout make_layout(int bits, int bn, int sl, int sc_bytes, int sc_bufs) {
+__host__ __device__ inline Layout make_layout(int bits, int bn, int mh, int sl, int sc_bytes,
+                                              int sc_bufs) {
   Layout L;
   const int raw_bytes = bn * BK * bits / 8;
   L.a = 0;
-  L.b = L.a + sl * kABytes;
+  L.b = L.a + sl * mh * kABytes;
   L.raw = L.b + kSB * bn * BK * 2;
   L.sc = L.raw + sl * raw_bytes;
   L.bar = (L.sc + sc_bufs * sc_bytes + 127) & ~127;
@@ -149,7 +152,7 @@ __device__ __forceinline__ uint4 dequant_int8_words(uint32_t w0, uint32_t w1, fl
   return out;
 }
 
-template <int BITS, int BN>
+template <int BITS, int BN, int MH>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s, const uint16_t *__restrict__ scales,
@@ -159,9 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
   constexpr int kRawBytes = BN * kRawRow;
   constexpr int kBBytes = BN * BK * 2;
-  constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+  constexpr int TM = BM * MH;                   // output rows per tile
+  constexpr int kAStage = MH * kABytes;         // X bytes per load stage
+  constexpr uint32_t kTmemCols = 2 * MH * BN;   // two accumulator sets of MH halves
+  static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
   constexpr uint32_t kIdesc = idesc_for(BN);
-  const Layout L = make_layout(BITS, BN, sl_stages, sc_bytes, sc_bufs);
+  const Layout L = make_layout(BITS, BN, MH, sl_stages, sc_bytes, sc_bufs);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_k = (K + BK - 1) / BK;
-  const int num_m = (M + BM - 1) / BM;
+  const int num_m = (M + TM - 1) / TM;
   // Work unit u covers output tile u / splits and K-stages [ks0, ks1) of split u % splits.
   const int num_units = num_m * ((N + BN - 1) / BN) * splits;
   const int kps = (num_k + splits - 1) / splits;
@@ -258,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::pdl_wait();
             waited = true;
           }
-          ptx::mbar_arrive_expect_tx(&sh.afull[s], kABytes);
-          ptx::tma_load_2d(smem + L.a + s * kABytes, &tm_x, &sh.afull[s], ks * BK, mb * BM);
+          ptx::mbar_arrive_expect_tx(&sh.afull[s], kAStage);
+          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.afull[s], ks * BK, mb * TM);
           amask |= 1u << s;
           apar = (apar & ~(1u << s)) | (ph << s);
           if (++s == SL) {
@@ -289,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d = tmem + static_cast<uint32_t>(ab * BN);
+        const uint32_t d = tmem + static_cast<uint32_t>(ab * MH * BN);
         for (int ks = ks0; ks < ks1; ++ks) {
           ok = ptx::mbar_wait_bounded(&sh.afull[s], ph, wait_limit, abort) &&
                ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort);
@@ -298,12 +304,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          // start-address field counts 16-byte units; K=16 bf16 = 32 bytes = 2 units
-          const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kABytes >> 4));
+          // start-address field counts 16-byte units; K=16 bf16 = 32 bytes = 2 units; the
+          // second 128-row half of the X tile starts kABytes further on
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kAStage >> 4));
           const uint64_t bd = bdesc0 + static_cast<uint64_t>(bs * (kBBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            ptx::tc_mma_f16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < MH; ++h)
+              ptx::tc_mma_f16(d + static_cast<uint32_t>(h * BN),
+                              ad + static_cast<uint64_t>(h * (kABytes >> 4)) + 2 * kk, bd + 2 * kk,
+                              kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
           mma_issued = true;
           ptx::tc_commit(&sh.lempty[s]);
           ptx::tc_commit(&sh.bempty[bs]);
@@ -326,12 +337,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_commit(&sh.drain);  // arrives once every MMA issued above has completed
     }
   } else if (warp < 2 + kDequantWarps) {
-    // ---- dequantisers: 512 threads, one job of E codes per stage each: row t % BN, part
-    //      t / BN of the stage's 64 codes (E = 32 at BN = 256, 16 at BN = 128) ----
+    // ---- dequantisers: 512 threads, one job of E codes per stage each: part t % P of row
+    //      t / P, P = 64 / E parts per row (E = 32 at BN = 256, 16 at BN = 128). A warp's lanes
+    //      cover 32 / P whole rows, so their raw-code loads are one contiguous range and their
+    //      swizzled B stores hit distinct bank groups ----
     constexpr int E = BN * BK / kDequantThreads;  // codes per job
     constexpr int CH = E / 8;                     // 16-byte B chunks per job
+    constexpr int P = BK / E;                     // jobs per row
     const int t = threadIdx.x - 64;
-    const int row = t % BN, part = t / BN;
+    const int row = t / P, part = t % P;
     const int spr = K >> 5;
     const int sw = row & 7;
     const int kbo = (part * E) >> 5;  // which 32-code block of the stage
@@ -440,11 +454,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::pdl_wait();
         waited = true;
       }
-      const int grow = mb * BM + q * 32 + lane;
       const int n0 = nb * BN;
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      for (int hc = 0; hc < MH * BN; hc += 16) {
+        const int h = hc / BN, c0 = hc - h * BN;
+        const int grow = mb * TM + h * BM + q * 32 + lane;
         uint32_t r[16];
-        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * BN + c0, r);
+        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * MH * BN + hc, r);
         ptx::tmem_ld_wait();
         if (grow < M) {
           float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
@@ -557,10 +572,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int BITS, int BN>
+template <int BITS, int BN, int MH>
 int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
               const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
-  auto kern = qgemm_tc_kernel<BITS, BN>;
+  auto kern = qgemm_tc_kernel<BITS, BN, MH>;
+  constexpr int TM = BM * MH;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
@@ -575,18 +591,18 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   const int64_t spr = w.k / 32;
   const bool sc_tma = spr % 8 == 0 && spr <= kTmaScaleCols;
   const int sc_bytes = sc_tma ? static_cast<int>((BN * spr * 2 + 127) & ~int64_t(127)) : 0;
-  const int stage = kABytes + BN * BK * BITS / 8;
+  const int stage = MH * kABytes + BN * BK * BITS / 8;
   auto stages_for = [&](int bufs) {
-    return std::min(kMaxSL, (kSmemMax - make_layout(BITS, BN, 0, sc_bytes, bufs).total) / stage);
+    return std::min(kMaxSL, (kSmemMax - make_layout(BITS, BN, MH, 0, sc_bytes, bufs).total) / stage);
   };
   int sc_bufs = sc_tma ? 2 : 1;
   if (sc_tma && stages_for(2) < 4) sc_bufs = 1;
   const int sl = stages_for(sc_bufs);
   if (sl < 2) return WOQ_ESHAPE;
-  const int smem = make_layout(BITS, BN, sl, sc_bytes, sc_bufs).total;
+  const int smem = make_layout(BITS, BN, MH, sl, sc_bytes, sc_bufs).total;
 
   CUtensorMap tm_x, tm_w, tm_s;
-  if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, BM,
+  if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, TM,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return WOQ_ECUDA;
   if (!make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
@@ -623,7 +639,7 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   // 2) the persistent GEMM: one CTA per SM (or per work unit, if fewer).
   float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + plan.xb);
   {
-    const int64_t tiles = ((m + BM - 1) / BM) * ((w.n + BN - 1) / BN) * plan.splits;
+    const int64_t tiles = ((m + TM - 1) / TM) * ((w.n + BN - 1) / BN) * plan.splits;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(tiles, dev.sm_count)), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -680,10 +696,13 @@ GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budg
   auto align = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };
   GemmPlan p;
   p.xb = align(static_cast<size_t>(m) * static_cast<size_t>(k) * 2);
-  const int64_t mt = (m + BM - 1) / BM;
   const int64_t num_k = (k + BK - 1) / BK;
-  // 128 x 256 tiles do twice the work per MMA instruction; prefer them when N allows.
-  p.bn = n >= 256 ? 256 : 128;
+  // Past one 128-row M tile, 256 x 128 tiles (two M halves sharing each dequantised weight
+  // tile) halve the dequantisation per FLOP. Otherwise 128 x 256 tiles, which do twice the
+  // work per MMA instruction, when N allows.
+  p.mh = m > 128 ? 2 : 1;
+  p.bn = p.mh == 1 && n >= 256 ? 256 : 128;
+  const int64_t mt = (m + 128 * p.mh - 1) / (128 * p.mh);
   int64_t tiles = mt * ((n + p.bn - 1) / p.bn);
   // Split K until the work units cover the SMs, keeping >= 4 K-stages per split; the splits
   // need FP32 partials in the workspace and a vectorisable Y (n % 4 == 0).
@@ -702,11 +721,14 @@ GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budg
 
 int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
                    const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
-  if (w.bits == 4)
-    return plan.bn == 256 ? launch_tc<4, 256>(X, m, w, Y, workspace, plan, s, dev)
-                          : launch_tc<4, 128>(X, m, w, Y, workspace, plan, s, dev);
-  return plan.bn == 256 ? launch_tc<8, 256>(X, m, w, Y, workspace, plan, s, dev)
-                        : launch_tc<8, 128>(X, m, w, Y, workspace, plan, s, dev);
+  if (w.bits == 4) {
+    if (plan.mh == 2) return launch_tc<4, 128, 2>(X, m, w, Y, workspace, plan, s, dev);
+    return plan.bn == 256 ? launch_tc<4, 256, 1>(X, m, w, Y, workspace, plan, s, dev)
+                          : launch_tc<4, 128, 1>(X, m, w, Y, workspace, plan, s, dev);
+  }
+  if (plan.mh == 2) return launch_tc<8, 128, 2>(X, m, w, Y, workspace, plan, s, dev);
+  return plan.bn == 256 ? launch_tc<8, 256, 1>(X, m, w, Y, workspace, plan, s, dev)
+                        : launch_tc<8, 128, 1>(X, m, w, Y, workspace, plan, s, dev);
 }
 
 int read_wait_timeout_flag(int clear, unsigned *value) {

@@ -51,7 +51,8 @@ int read_gemv_tc_timeout_flag(int clear, unsigned *value);
 // How the tensor-core path runs a problem: tile width, K-splits and workspace layout
 // ([bf16 copy of X][FP32 partials of the splits], each 256-byte aligned).
 struct GemmPlan {
-  int bn = 128;
+  int bn = 128;   // output columns per tile
+  int mh = 1;     // 128-row M halves per tile (2: both share each dequantised weight tile)
   int splits = 1;
   size_t xb = 0, part = 0, total = 0;
 };
