@@ -8,13 +8,14 @@
 //   warp 0        producer: bulk tensor copies (TMA, no multicast) of the bf16 X tile
 //                 (128B-swizzled, 128 * MH rows) and the raw code tile into a ring of SL load
 //                 stages, and of each output tile's [BN, K/32] scale tile into a double buffer
-//   warp 1        TMEM owner; one thread issues tcgen05.mma (M=128, N=BN, K=16, bf16 x
-//                 bf16 -> f32), one per 128-row half of the tile, into one of two accumulator
-//                 sets and commits completions
+//   warp 1        TMEM owner; one thread issues tcgen05.mma (K=16, bf16 x bf16 -> f32) into
+//                 one of two accumulator sets and commits completions: M=128 activation rows x
+//                 N=BN for MH = 1; for MH = 2 the operands swap, M=128 weight rows x N=256
+//                 activation rows
 //   warps 2..17   dequantisers: raw codes + binary16 scales -> bf16(scale * code) written
 //                 into a short ring of B tiles in the 128B-swizzled K-major layout that the
-//                 MMA's shared-memory descriptor names; with MH = 2 each B tile feeds both
-//                 halves, so the dequantisation per FLOP is halved
+//                 MMA's shared-memory descriptor names; with MH = 2 each weight tile meets 256
+//                 activation rows, so the dequantisation per FLOP is halved
 //   warps 18..21  epilogue: tcgen05.ld of the finished accumulators -> FP32 Y, while the MMA
 //                 thread already fills the other set with the next tile
 // Every mbarrier wait is bounded. A wait that gives up records the event in a device flag
@@ -50,9 +51,9 @@ constexpr long long kDrainLimit = 1LL << 31;                    // cycles (~1 s)
 constexpr long long kDefaultWaitLimit = 1LL << 32;              // cycles (~2 s)
 constexpr int kSmemMax = 227 * 1024;
 
-// Instruction descriptor: D f32, A/B bf16, both K-major, N = bn, M = BM.
-__host__ __device__ constexpr uint32_t idesc_for(int bn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) |
+// Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_for(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(BM >> 4) << 24);
 }
 
@@ -162,11 +163,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
   constexpr int kRawBytes = BN * kRawRow;
   constexpr int kBBytes = BN * BK * 2;
-  constexpr int TM = BM * MH;                   // output rows per tile
+  constexpr int TM = BM * MH;                   // output rows (activation rows) per tile
   constexpr int kAStage = MH * kABytes;         // X bytes per load stage
-  constexpr uint32_t kTmemCols = 2 * MH * BN;   // two accumulator sets of MH halves
+  // MH = 1: the MMA's A is the X tile and B the weight tile; the accumulator holds
+  // [128 activation rows x BN]. MH = 2: the roles swap, A = the 128-row weight tile and
+  // B = the 256-row X tile, so one M=128, N=256 MMA per K-step covers the whole tile (long
+  // MMAs keep the tensor pipe fed between stages); the accumulator holds [BN = 128 weight
+  // rows x 256 activation rows].
+  static_assert(MH == 1 || BN == BM, "swapped tiles need 128 weight rows");
+  constexpr int kAccCols = MH == 2 ? TM : BN;   // accumulator columns per set
+  constexpr uint32_t kTmemCols = 2 * kAccCols;  // two accumulator sets
   static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
-  constexpr uint32_t kIdesc = idesc_for(BN);
+  constexpr uint32_t kIdesc = idesc_for(MH == 2 ? TM : BN);
   const Layout L = make_layout(BITS, BN, MH, sl_stages, sc_bytes, sc_bufs);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -295,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d = tmem + static_cast<uint32_t>(ab * MH * BN);
+        const uint32_t d = tmem + static_cast<uint32_t>(ab * kAccCols);
         for (int ks = ks0; ks < ks1; ++ks) {
           ok = ptx::mbar_wait_bounded(&sh.afull[s], ph, wait_limit, abort) &&
                ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort);
@@ -309,12 +317,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kAStage >> 4));
           const uint64_t bd = bdesc0 + static_cast<uint64_t>(bs * (kBBytes >> 4));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-#pragma unroll
-            for (int h = 0; h < MH; ++h)
-              ptx::tc_mma_f16(d + static_cast<uint32_t>(h * BN),
-                              ad + static_cast<uint64_t>(h * (kABytes >> 4)) + 2 * kk, bd + 2 * kk,
-                              kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if constexpr (MH == 2)
+              ptx::tc_mma_f16(d, bd + 2 * kk, ad + 2 * kk, kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
+            else
+              ptx::tc_mma_f16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
+          }
           mma_issued = true;
           ptx::tc_commit(&sh.lempty[s]);
           ptx::tc_commit(&sh.bempty[bs]);
@@ -455,11 +463,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         waited = true;
       }
       const int n0 = nb * BN;
-      for (int hc = 0; hc < MH * BN; hc += 16) {
-        const int h = hc / BN, c0 = hc - h * BN;
-        const int grow = mb * TM + h * BM + q * 32 + lane;
+      if constexpr (MH == 2) {
+        // TMEM lane = weight row n, column = activation row m: for each column the warp's
+        // 32 lanes store 32 consecutive floats of one Y row.
+        const int n = n0 + q * 32 + lane;
+        for (int c0 = 0; c0 < TM && mb * TM + c0 < M; c0 += 16) {
+          uint32_t r[16];
+          ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols + c0, r);
+          ptx::tmem_ld_wait();
+          if (n < N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int m = mb * TM + c0 + j;
+              if (m < M) out[static_cast<size_t>(m) * N + n] = __uint_as_float(r[j]);
+            }
+          }
+        }
+      }
+      for (int c0 = 0; MH == 1 && c0 < BN; c0 += 16) {
+        const int grow = mb * TM + q * 32 + lane;
         uint32_t r[16];
-        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * MH * BN + hc, r);
+        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols + c0, r);
         ptx::tmem_ld_wait();
         if (grow < M) {
           float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
