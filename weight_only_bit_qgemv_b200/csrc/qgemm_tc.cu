@@ -40,7 +40,10 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;              // bf16 elements per stage = one 128-byte swizzle row
 constexpr int kMaxSL = 8;           // load stages (X tile + raw code tile)
-constexpr int kSB = 2;              // dequantised B tiles
+constexpr int kMaxSB = 4;           // dequantised weight tiles (ring), at most
+// Weight-tile ring depth: 4 for 128-row tiles (the dequantisers then run two stages ahead
+// of the MMAs instead of waiting on each stage's completion), 2 for 256-row tiles.
+__host__ __device__ constexpr int sb_for(int bn) { return bn == 128 ? 4 : 2; }
 constexpr int kTmaScaleCols = 128;  // scale tile copied by TMA when K/32 <= this (and % 8 == 0)
 constexpr int kDequantWarps = 16;  // four per scheduler: each warp's chain is latency-bound
 constexpr int kDequantThreads = kDequantWarps * 32;
@@ -50,6 +53,10 @@ constexpr int kABytes = BM * BK * 2;                            // 16 KB
 constexpr long long kDrainLimit = 1LL << 31;                    // cycles (~1 s)
 constexpr long long kDefaultWaitLimit = 1LL << 32;              // cycles (~2 s)
 constexpr int kSmemMax = 227 * 1024;
+// The single-lane roles (producer, MMA issuer) and the epilogue wait with a suspend hint:
+// back-to-back polling by them takes issue slots from the dequantising warps that share
+// their schedulers.
+constexpr uint32_t kRoleSleepNs = 200;
 
 // Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_for(int n) {
@@ -60,11 +67,10 @@ __host__ __device__ constexpr uint32_t idesc_for(int n) {
 long long g_wait_limit_cycles = 0;  // test hook: > 0 wait limit, < 0 inject a stuck wait
 
 struct Shared {
-  uint64_t afull[kMaxSL];   // X tile landed (TMA bytes)
-  uint64_t wfull[kMaxSL];   // raw code tile landed (TMA bytes)
+  uint64_t wfull[kMaxSL];   // raw code tile and X tile landed (TMA bytes)
   uint64_t lempty[kMaxSL];  // load stage free: MMA commit + one arrival per dequant warp
-  uint64_t bfull[kSB];      // B tile written (one arrival per dequant warp)
-  uint64_t bempty[kSB];     // B tile read by the MMAs (commit)
+  uint64_t bfull[kMaxSB];   // B tile written (one arrival per dequant warp)
+  uint64_t bempty[kMaxSB];  // B tile read by the MMAs (commit)
   uint64_t sfull[2];        // scale tile landed (TMA bytes)
   uint64_t sempty[2];       // scale tile done with (one arrival per dequant warp)
   uint64_t accfull[2];      // accumulator complete (commit)
@@ -85,7 +91,7 @@ __host__ __device__ inline Layout make_layout(int bits, int bn, int mh, int sl, 
   const int raw_bytes = bn * BK * bits / 8;
   L.a = 0;
   L.b = L.a + sl * mh * kABytes;
-  L.raw = L.b + kSB * bn * BK * 2;
+  L.raw = L.b + sb_for(bn) * bn * BK * 2;
   L.sc = L.raw + sl * raw_bytes;
   L.bar = (L.sc + sc_bufs * sc_bytes + 127) & ~127;
   L.total = L.bar + static_cast<int>(sizeof(Shared)) + 1024;  // + base alignment slack
@@ -163,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
   constexpr int kRawBytes = BN * kRawRow;
   constexpr int kBBytes = BN * BK * 2;
+  constexpr int kSB = sb_for(BN);              // weight-tile ring depth
   constexpr int TM = BM * MH;                   // output rows (activation rows) per tile
   constexpr int kAStage = MH * kABytes;         // X bytes per load stage
   // MH = 1: the MMA's A is the X tile and B the weight tile; the accumulator holds
@@ -194,7 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SL; ++s) {
-      ptx::mbar_init(&sh.afull[s], 1);
       ptx::mbar_init(&sh.wfull[s], 1);
       ptx::mbar_init(&sh.lempty[s], 1 + kDequantWarps);  // MMA commit + dequant warps
     }
@@ -229,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // producer bookkeeping for the drain: slots issued at least once, and the parity of
   // their last issue
-  uint32_t wmask = 0, wpar = 0, amask = 0, apar = 0, smask = 0, spar = 0;
+  uint32_t wmask = 0, wpar = 0, smask = 0, spar = 0;
   bool mma_issued = false;
 
   if (warp == 0) {
@@ -245,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int mb = tile % num_m, nb = tile / num_m;
         const int ks0 = sp * kps, ks1 = min(num_k, ks0 + kps);
         if (sc_tma) {
-          if (!ptx::mbar_wait_bounded(&sh.sempty[sb], sph ^ 1, wait_limit, abort)) {
+          if (!ptx::mbar_wait_bounded(&sh.sempty[sb], sph ^ 1, wait_limit, abort, kRoleSleepNs)) {
             record_timeout(abort);
             break;
           }
@@ -259,12 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         for (int ks = ks0; ks < ks1; ++ks) {
-          if (!ptx::mbar_wait_bounded(&sh.lempty[s], ph ^ 1, wait_limit, abort)) {
+          if (!ptx::mbar_wait_bounded(&sh.lempty[s], ph ^ 1, wait_limit, abort, kRoleSleepNs)) {
             record_timeout(abort);
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(&sh.wfull[s], kRawBytes);
+          // Both copies of the stage complete on one barrier. The dequantisers wait on it and
+          // only then mark their weight tile ready, so the MMA thread waits once per stage.
+          ptx::mbar_arrive_expect_tx(&sh.wfull[s], kRawBytes + kAStage);
           ptx::tma_load_2d(smem + L.raw + s * kRawBytes, &tm_w, &sh.wfull[s], ks * kRawRow, nb * BN);
           wmask |= 1u << s;
           wpar = (wpar & ~(1u << s)) | (ph << s);
@@ -272,10 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::pdl_wait();
             waited = true;
           }
-          ptx::mbar_arrive_expect_tx(&sh.afull[s], kAStage);
-          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.afull[s], ks * BK, mb * TM);
-          amask |= 1u << s;
-          apar = (apar & ~(1u << s)) | (ph << s);
+          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.wfull[s], ks * BK, mb * TM);
           if (++s == SL) {
             s = 0;
             ph ^= 1;
@@ -298,15 +303,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0, bph = 0, aph = 0;
       for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
         const int ks0 = (u - (u / splits) * splits) * kps, ks1 = min(num_k, ks0 + kps);
-        if (!ptx::mbar_wait_bounded(&sh.accempty[ab], aph ^ 1, wait_limit, abort)) {
+        if (!ptx::mbar_wait_bounded(&sh.accempty[ab], aph ^ 1, wait_limit, abort, kRoleSleepNs)) {
           record_timeout(abort);
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(ab * kAccCols);
         for (int ks = ks0; ks < ks1; ++ks) {
-          ok = ptx::mbar_wait_bounded(&sh.afull[s], ph, wait_limit, abort) &&
-               ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort);
+          // bfull completes after every dequantiser has seen this stage's copies land (X and
+          // the raw codes share wfull), so it covers the X tile as well.
+          ok = ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort);
           if (!ok) {
             record_timeout(abort);
             break;
@@ -453,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mb = tile % num_m, nb = tile / num_m;
       // One split writes Y; several write FP32 partials [split][M][N] for the reduction.
       float *out = splits == 1 ? Y : partials + static_cast<size_t>(sp) * M * N;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.accfull[ab], aph, wait_limit, abort))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.accfull[ab], aph, wait_limit, abort, kRoleSleepNs))) {
         record_timeout(abort);
         break;
       }
@@ -463,14 +469,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         waited = true;
       }
       const int n0 = nb * BN;
-      if constexpr (MH == 2) {
-        // TMEM lane = weight row n, column = activation row m: for each column the warp's
-        // 32 lanes store 32 consecutive floats of one Y row.
-        const int n = n0 + q * 32 + lane;
-        for (int c0 = 0; c0 < TM && mb * TM + c0 < M; c0 += 16) {
-          uint32_t r[16];
-          ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols + c0, r);
-          ptx::tmem_ld_wait();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
+      // 16-column chunks, software-pipelined: the next chunk's TMEM load is in flight while
+      // this one is stored (two register buffers, each waited for before use).
+      const int ncols = MH == 2 ? min(TM, M - mb * TM) : BN;
+      const int nchunks = (ncols + 15) / 16;
+      auto store_chunk = [&](const uint32_t (&r)[16], int c) {
+        const int c0 = 16 * c;
+        if constexpr (MH == 2) {
+          // TMEM lane = weight row n, column = activation row m: for each column the warp's
+          // 32 lanes store 32 consecutive floats of one Y row.
+          const int n = n0 + q * 32 + lane;
           if (n < N) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -478,26 +487,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (m < M) out[static_cast<size_t>(m) * N + n] = __uint_as_float(r[j]);
             }
           }
-        }
-      }
-      for (int c0 = 0; MH == 1 && c0 < BN; c0 += 16) {
-        const int grow = mb * TM + q * 32 + lane;
-        uint32_t r[16];
-        ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols + c0, r);
-        ptx::tmem_ld_wait();
-        if (grow < M) {
-          float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
-          if (vec && n0 + c0 + 16 <= N) {
+        } else {
+          const int grow = mb * TM + q * 32 + lane;
+          if (grow < M) {
+            float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
+            if (vec && n0 + c0 + 16 <= N) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              reinterpret_cast<float4 *>(yr)[v] =
-                  make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                              __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          } else {
+              for (int v = 0; v < 4; ++v)
+                reinterpret_cast<float4 *>(yr)[v] =
+                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            } else {
 #pragma unroll
-            for (int v = 0; v < 16; ++v)
-              if (n0 + c0 + v < N) yr[v] = __uint_as_float(r[v]);
+              for (int v = 0; v < 16; ++v)
+                if (n0 + c0 + v < N) yr[v] = __uint_as_float(r[v]);
+            }
           }
+        }
+      };
+      uint32_t ra[16], rb[16];
+      ptx::tmem_ld_32x32b_x16(tb, ra);
+      ptx::tmem_ld_wait(ra);
+      for (int c = 0; c < nchunks; c += 2) {  // trip counts are warp-uniform
+        if (c + 1 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 1), rb);
+        store_chunk(ra, c);
+        if (c + 1 < nchunks) {
+          ptx::tmem_ld_wait(rb);
+          if (c + 2 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 2), ra);
+          store_chunk(rb, c + 1);
+          if (c + 2 < nchunks) ptx::tmem_ld_wait(ra);
         }
       }
       ptx::tc_fence_before();
@@ -518,8 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < SL; ++i) {
       if ((wmask >> i) & 1)
         ptx::mbar_wait_bounded(&sh.wfull[i], (wpar >> i) & 1, kDrainLimit, &no_abort);
-      if ((amask >> i) & 1)
-        ptx::mbar_wait_bounded(&sh.afull[i], (apar >> i) & 1, kDrainLimit, &no_abort);
     }
     for (int i = 0; i < sc_bufs; ++i)
       if ((smask >> i) & 1)

@@ -493,7 +493,8 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
       for (int tile = blockIdx.x, i = 0; tile < full_tiles; tile += gridDim.x, ++i) {
         const int s = i % stages;
         const int round = i / stages;
-        if (round > 0 && !ptx::mbar_wait_bounded(&sh.empty[s], (round - 1) & 1, kGemvWaitLimit, abort)) {
+        if (round > 0 && !ptx::mbar_wait_bounded(&sh.empty[s], (round - 1) & 1, kGemvWaitLimit, abort,
+                                                 NW == 8 ? 1000u : 0u)) {
           gemv_record_timeout(abort);
           break;
         }
@@ -542,8 +543,11 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     const bool staged = tile < full_tiles;
     const int s = i % stages;
     // The outcome is made warp-uniform: shuffles and the elected arrival follow.
+    // Bandwidth-bound launches (NW = 8) let waiting warps sleep so that the computing ones
+    // get the issue slots; latency-bound ones (NW = 16) poll.
     if (staged && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.full[s], (i / stages) & 1,
-                                                                   kGemvWaitLimit, abort))) {
+                                                                   kGemvWaitLimit, abort,
+                                                                   NW == 8 ? 1000u : 0u))) {
       gemv_record_timeout(abort);
       break;
     }
