@@ -478,13 +478,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = 16 * c;
         if constexpr (MH == 2) {
           // TMEM lane = weight row n, column = activation row m: for each column the warp's
-          // 32 lanes store 32 consecutive floats of one Y row.
+          // 32 lanes store 32 consecutive floats of one Y row. The row pointer advances by
+          // N per column; full chunks skip the row check.
           const int n = n0 + q * 32 + lane;
+          const int mrem = M - (mb * TM + c0);
+          float *p = out + static_cast<size_t>(mb * TM + c0) * N + n;
           if (n < N) {
+            if (mrem >= 16) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int m = mb * TM + c0 + j;
-              if (m < M) out[static_cast<size_t>(m) * N + n] = __uint_as_float(r[j]);
+              for (int j = 0; j < 16; ++j, p += N) *p = __uint_as_float(r[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j, p += N)
+                if (j < mrem) *p = __uint_as_float(r[j]);
             }
           }
         } else {
