@@ -129,6 +129,23 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
                void *stream);
 
 /*
+ * qgemv_argmax -- greedy pick over a GEMV's outputs without writing them: for each activation
+ * row i, idx[i] = the smallest j with y[i, j] = max over j of y[i, j], and val[i] = that
+ * maximum, where y = x . W_hat^T is computed exactly as qgemv's CUDA-core form computes it.
+ * Meant for the tied lm_head at decode under greedy decoding (the soniqo guide, Russian
+ * edition, "Заметки реализации": its runtime decodes greedily): the 151,936 logits are
+ * never written. A NaN output counts as the maximum. Deterministic.
+ *   x    device, [m, k] float32 row-major, 16-byte aligned, 1 <= m <= 8
+ *   w    host pointer to the weight descriptor (read during the call only)
+ *   idx  device, [m] int64, 8-byte aligned; used as scratch during the call, then the index
+ *   val  device, [m] float32; the maximum
+ * Limits: k <= 8192 and n < 2^31. Errors: as qgemv, and WOQ_ESHAPE for shapes the fused
+ * kernel does not cover.
+ */
+int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, float *val,
+                 void *stream);
+
+/*
  * Bytes of device workspace qgemm needs for (m, w, path); 0 if none. Returns 0 for
  * invalid arguments too (qgemm itself reports those).
  */

@@ -26,5 +26,7 @@ from .woq_ref import (  # noqa: F401
     qgemv_ref,
     qgemm_ref,
     qgemm_bf16_ref,
+    greedy_ref,
+    qgemv_argmax_ref,
     bf16_round,
 )

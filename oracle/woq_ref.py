@@ -183,6 +183,24 @@ def qgemm_bf16_ref(X: np.ndarray, packed: np.ndarray, scale_bits: np.ndarray, bi
     return matmul_ref(bf16_round(X), bf16_round(W_hat))
 
 
+def greedy_ref(Y: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Greedy decoding's pick over each row of outputs Y [M, N]: the first index of the
+    row maximum, and that maximum ("MOSS Transcribe Diarize 0.9B", soniqo Russian guide,
+    "Implementation notes": the runtime decodes greedily). NaN counts as the maximum.
+    """
+    Y = np.atleast_2d(np.asarray(Y, dtype=np.float64))
+    idx = np.empty(Y.shape[0], dtype=np.int64)
+    for i, row in enumerate(Y):
+        nan = np.flatnonzero(np.isnan(row))
+        idx[i] = nan[0] if nan.size else int(np.argmax(row))
+    return idx, Y[np.arange(Y.shape[0]), idx]
+
+
+def qgemv_argmax_ref(X: np.ndarray, packed: np.ndarray, scale_bits: np.ndarray, bits: int):
+    """Greedy pick over the exact outputs: greedy_ref(qgemv_ref(...))."""
+    return greedy_ref(qgemv_ref(X, packed, scale_bits, bits))
+
+
 def fsum_dot(x_row: np.ndarray, w_row: np.ndarray) -> float:
     """Correctly rounded dot product of two float64 vectors (math.fsum), for tiny cases."""
     return math.fsum(float(a) * float(b) for a, b in zip(x_row, w_row))

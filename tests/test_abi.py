@@ -68,6 +68,13 @@ def test_argument_checks_return_before_touching_a_device():
     assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, 3, None) == _lib.WOQ_EINVAL
     assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, -1, None) == _lib.WOQ_EINVAL
     assert L.qgemv_path(ok_ptr, 65, ctypes.byref(w), ok_ptr, _lib.WOQ_GEMV_SPLIT_TC, None) == _lib.WOQ_EINVAL
+    # qgemv_argmax: 1 <= m <= 8, k <= 8192, idx 8-byte aligned
+    assert L.qgemv_argmax(ok_ptr, 0, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv_argmax(ok_ptr, 9, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv_argmax(ok_ptr, 1, ctypes.byref(w), None, ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv_argmax(ok_ptr, 1, ctypes.byref(w), ok_ptr + 4, ok_ptr, None) == _lib.WOQ_EALIGN
+    wide = _w(k=16384, packed=ok_ptr, scales=ok_ptr)
+    assert L.qgemv_argmax(ok_ptr, 1, ctypes.byref(wide), ok_ptr, ok_ptr, None) == _lib.WOQ_ESHAPE
     # bf16 path: workspace checked before the device
     need = L.qgemm_workspace_bytes(256, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC)
     assert need == 256 * 64 * 2

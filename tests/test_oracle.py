@@ -350,3 +350,33 @@ def test_bf16_reading_error_is_within_the_tolerance_budget():
         e = oracle.qgemm_bf16_ref(X, p, sb, bits) - oracle.qgemv_ref(X, p, sb, bits)
         rel = np.linalg.norm(e) / np.linalg.norm(oracle.qgemv_ref(X, p, sb, bits))
         assert 1e-4 < rel < 1e-2
+
+
+# ---- greedy pick (qgemv_argmax reference) ----
+
+def test_greedy_ref_first_index_among_ties_and_nan():
+    Y = np.array([[1.0, 3.0, 3.0, -2.0],
+                  [-5.0, -1.0, -1.0, -7.0],
+                  [0.0, np.nan, 9.0, np.nan],
+                  [2.0, 2.0, 2.0, 2.0]])
+    idx, val = oracle.greedy_ref(Y)
+    assert idx.tolist() == [1, 1, 1, 0]
+    assert val[0] == 3.0 and val[1] == -1.0 and np.isnan(val[2]) and val[3] == 2.0
+
+
+def test_qgemv_argmax_ref_on_a_hand_built_weight():
+    # every block's max |w| is 7 = qmax for int4, so every scale is exactly 1 and the codes
+    # equal the weights; y_j = c_j * x_0 with c = (1, 7, -7, 7, 3) (x_1 = 0)
+    K = 32
+    W = np.zeros((5, K), dtype=np.float32)
+    W[:, 0] = [1.0, 7.0, -7.0, 7.0, 3.0]
+    W[:, 1] = 7.0
+    q, s = oracle.quantise(W, 4)
+    assert np.all(oracle.fp16_bits_to_float(s) == 1.0)
+    p = oracle.pack(q, 4)
+    x = np.zeros((1, K), dtype=np.float32); x[0, 0] = 2.0
+    idx, val = oracle.qgemv_argmax_ref(x, p, s, 4)
+    assert idx.tolist() == [1] and val.tolist() == [14.0]   # tie with j = 3: first index
+    x[0, 0] = -2.0                                            # now -7 * -2 = 14 at j = 2
+    idx, val = oracle.qgemv_argmax_ref(x, p, s, 4)
+    assert idx.tolist() == [2] and val.tolist() == [14.0]

@@ -33,6 +33,7 @@ __all__ = [
     "qpack",
     "pack",
     "qgemv",
+    "qgemv_argmax",
     "qgemm",
     "qgemm_workspace_bytes",
     "device_status",
@@ -115,6 +116,20 @@ def qgemv(
     rc = _lib.lib().qgemv_path(_ptr(x), m, ctypes.byref(d), _ptr(out), _GEMV_PATHS[path], _stream(stream))
     _lib.check(rc, "qgemv")
     return out
+
+
+def qgemv_argmax(x: torch.Tensor, w: PackedWeight, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Per activation row, the index (smallest among ties) and value of the largest output of
+    x . W_hat^T, without writing the outputs (C ABI ``qgemv_argmax``); 1 <= m <= 8."""
+    if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
+    m = x.shape[0]
+    idx = torch.empty(m, dtype=torch.int64, device=x.device)
+    val = torch.empty(m, dtype=torch.float32, device=x.device)
+    d = w.desc()
+    rc = _lib.lib().qgemv_argmax(_ptr(x), m, ctypes.byref(d), _ptr(idx), _ptr(val), _stream(stream))
+    _lib.check(rc, "qgemv_argmax")
+    return idx, val
 
 
 def qgemm_workspace_bytes(m: int, w: PackedWeight, path: str = "auto") -> int:

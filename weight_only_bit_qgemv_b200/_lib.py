@@ -30,6 +30,7 @@ EXPORTS = (
     "qpack",
     "qgemv",
     "qgemv_path",
+    "qgemv_argmax",
     "qgemm_workspace_bytes",
     "qgemm",
     "qgemm_bf16_noalloc",
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
     L.qgemv.restype = ctypes.c_int
     L.qgemv_path.argtypes = [vp, c_i64, wp, vp, c_i32, vp]
     L.qgemv_path.restype = ctypes.c_int
+    L.qgemv_argmax.argtypes = [vp, c_i64, wp, vp, vp, vp]
+    L.qgemv_argmax.restype = ctypes.c_int
     L.qgemm_workspace_bytes.argtypes = [c_i64, wp, c_i32]
     L.qgemm_workspace_bytes.restype = ctypes.c_size_t
     L.qgemm.argtypes = [vp, c_i64, wp, vp, c_i32, vp, ctypes.c_size_t, vp]

@@ -99,6 +99,20 @@ int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream
   return qgemv_path(x, m, w, y, WOQ_GEMV_AUTO, stream);
 }
 
+int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, float *val,
+                 void *stream) {
+  int rc = woq::check_weight(w);
+  if (rc != WOQ_OK) return rc;
+  if (!x || !idx || !val) return WOQ_EINVAL;
+  if (m < 1 || m > 8) return WOQ_EINVAL;
+  if (w->k > 8192 || w->n >= (int64_t(1) << 31)) return WOQ_ESHAPE;
+  if (!woq::aligned(x, 16) || !woq::aligned(idx, 8) || !woq::aligned(val, 4)) return WOQ_EALIGN;
+  DevInfo dev;
+  rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  return woq::launch_gemv_argmax(x, m, *w, idx, val, static_cast<cudaStream_t>(stream), dev);
+}
+
 // SM count the tensor-core plan is made for: the current device's, or 0 (no K-splits) when
 // no device can be queried, so that sizing never fails.
 static int plan_sm_count() {

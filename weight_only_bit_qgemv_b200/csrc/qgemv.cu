@@ -20,6 +20,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 #include <unordered_map>
 
 #include "ptx.cuh"
@@ -442,6 +443,7 @@ constexpr long long kGemvDrainLimit = 1LL << 31;  // cycles (~1 s)
 struct BulkShared {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
+  unsigned long long amax[8];  // argmax mode: this CTA's best key per activation row
   int abort;
 };
 static_assert(sizeof(BulkShared) <= kBulkHeader, "header too small");
@@ -451,11 +453,23 @@ __device__ __forceinline__ void gemv_record_timeout(volatile int *abort) {
   atomicOr(&g_gemv_timeout_flag, 1u);
 }
 
-template <int BITS, int MT, int RW, int NW>
+// Argmax keys: the output's bits mapped to an unsigned order that agrees with the float
+// order, every NaN (of either sign) above +inf, then the complement of the row so that ties
+// go to the smaller row.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int row) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t o = (v != v) ? 0xFFFFFFFFu : (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(o) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(row));
+}
+
+// AMAX = false: y[m, n] is written. AMAX = true: nothing is written to y; for each activation
+// row, the CTA's largest key over its outputs goes into keys[row] by a 64-bit atomicMax.
+template <int BITS, int MT, int RW, int NW, bool AMAX = false>
 __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
                      const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n,
-                     int k, int stages, int stage_bytes, int x_bytes) {
+                     int k, int stages, int stage_bytes, int x_bytes,
+                     unsigned long long *__restrict__ keys = nullptr) {
   constexpr int kBulkWarps = NW;
   constexpr int TR = kBulkWarps * RW;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -482,6 +496,7 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
       ptx::mbar_init(&sh.empty[s], kBulkWarps);
     }
     sh.abort = 0;
+    for (int mm = 0; mm < MT; ++mm) sh.amax[mm] = 0ull;
     ptx::fence_mbar_init();
   }
   __syncthreads();
@@ -538,6 +553,7 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kBulkWarps * 32) : "memory");
   ptx::pdl_launch_dependents();
+  unsigned long long best = 0ull;  // argmax mode: this lane's best key (activation row lane % MT)
 
   for (int tile = blockIdx.x, i = 0; tile < num_tiles; tile += gridDim.x, ++i) {
     const bool staged = tile < full_tiles;
@@ -589,8 +605,29 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     for (int r = 0; r < RW; ++r)
 #pragma unroll
       for (int mm = 0; mm < MT; ++mm)
-        if (lane == r * MT + mm && row0 + r < n && m0 + mm < m)
-          y[static_cast<size_t>(m0 + mm) * n + row0 + r] = acc[r][mm];
+        if (lane == r * MT + mm && row0 + r < n && m0 + mm < m) {
+          if constexpr (AMAX) {
+            const unsigned long long key = argmax_key(acc[r][mm], row0 + r);
+            best = key > best ? key : best;
+          } else
+            y[static_cast<size_t>(m0 + mm) * n + row0 + r] = acc[r][mm];
+        }
+  }
+  if constexpr (AMAX) {
+    // Lanes l and l ^ d with d >= MT hold keys of the same activation row (lane % MT): reduce
+    // over them, then one shared atomic per warp and row.
+#pragma unroll
+    for (int d = 16; d >= MT; d >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, d);
+      best = o > best ? o : best;
+    }
+    if (lane < MT) atomicMax(&sh.amax[lane], best);
+    // Every compute warp reaches this barrier (a warp that gave up on a wait leaves its loop
+    // and arrives here too); then one thread publishes the CTA's keys.
+    asm volatile("bar.sync 1, %0;" ::"n"(kBulkWarps * 32) : "memory");
+    if (tid == 0)
+      for (int mm = 0; mm < MT; ++mm)
+        if (m0 + mm < m) atomicMax(&keys[m0 + mm], sh.amax[mm]);
   }
 }
 
@@ -700,10 +737,11 @@ int pick_ru(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
 constexpr size_t kStageTarget = 20 * 1024;   // bytes per ring stage to aim for
 constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
 
-template <int BITS, int MT, int RW, int NW>
+template <int BITS, int MT, int RW, int NW, bool AMAX = false>
 int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
-                  const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes) {
-  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW>;
+                  const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes,
+                  unsigned long long *keys = nullptr) {
+  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW, AMAX>;
   constexpr int kBulkThreads = bulk_threads(NW);
   constexpr int TR = NW * RW;
   const int64_t num_tiles = (w.n + TR - 1) / TR;
@@ -734,7 +772,7 @@ int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cuda
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, w.packed, w.scales, y, static_cast<int>(m),
                                            static_cast<int>(w.n), static_cast<int>(w.k),
                                            static_cast<int>(stages), static_cast<int>(stage_bytes),
-                                           static_cast<int>(x_bytes));
+                                           static_cast<int>(x_bytes), keys);
   if (e != cudaSuccess) return WOQ_ECUDA;
   count_launches(1);
   return WOQ_OK;
@@ -747,22 +785,26 @@ inline int bulk_rows_per_warp(int nw, int rw_max, size_t row_total) {
   return rw;
 }
 
-template <int BITS, int MT, int NW>
+template <int BITS, int MT, int NW, bool AMAX = false>
 int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
-                   const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes) {
+                   const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes,
+                   unsigned long long *keys = nullptr) {
   // More rows per warp only where registers allow.
   int rw = bulk_rows_per_warp(NW, NW == 16 ? 2 : MT <= 2 ? 4 : 2, row_total);
   const size_t stage_bytes = (static_cast<size_t>(NW) * rw * row_total + 127) & ~size_t(127);
   if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return 1;
   if (w.n < NW * rw) rw = 1;  // tiny n: one row per warp, all from global memory
   if constexpr (MT <= 2 && NW == 8) {
-    if (rw == 4) return launch_bulk_t<BITS, MT, 4, NW>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+    if (rw == 4)
+      return launch_bulk_t<BITS, MT, 4, NW, AMAX>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
   }
   if constexpr (NW == 8 || MT == 1) {
-    if (rw >= 2) return launch_bulk_t<BITS, MT, 2, NW>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes);
+    if (rw >= 2)
+      return launch_bulk_t<BITS, MT, 2, NW, AMAX>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
   }
-  return launch_bulk_t<BITS, MT, 1, NW>(x, m, w, y, s, dev, pdl,
-                                        (static_cast<size_t>(NW) * row_total + 127) & ~size_t(127), x_bytes);
+  return launch_bulk_t<BITS, MT, 1, NW, AMAX>(x, m, w, y, s, dev, pdl,
+                                              (static_cast<size_t>(NW) * row_total + 127) & ~size_t(127),
+                                              x_bytes, keys);
 }
 
 template <int BITS, int MT>
@@ -805,6 +847,43 @@ int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
   }
 }
 
+// qgemv_argmax's first and last steps: zero the keys; turn each key back into
+// (row, output). Both wait on the preceding grid before touching memory.
+__global__ void __launch_bounds__(32) argmax_init_kernel(unsigned long long *keys, int m) {
+  ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
+  if (static_cast<int>(threadIdx.x) < m) keys[threadIdx.x] = 0ull;
+}
+
+__global__ void __launch_bounds__(32) argmax_final_kernel(unsigned long long *keys, float *val,
+                                                          int m) {
+  ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
+  const int i = threadIdx.x;
+  if (i >= m) return;
+  const unsigned long long key = keys[i];
+  const uint32_t o = static_cast<uint32_t>(key >> 32);
+  const uint32_t b = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
+  val[i] = __uint_as_float(b);
+  reinterpret_cast<long long *>(keys)[i] =
+      static_cast<long long>(0xFFFFFFFFu - static_cast<uint32_t>(key & 0xFFFFFFFFull));
+}
+
+template <int BITS>
+int argmax_bulk(const float *x, int64_t m, const woq_weight &w, unsigned long long *keys,
+                cudaStream_t s, const DevInfo &dev) {
+  const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
+  auto go = [&](auto mt_tag) -> int {
+    constexpr int MT = decltype(mt_tag)::value;
+    const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
+    return launch_bulk_nw<BITS, MT, 8, true>(x, m, w, nullptr, s, dev, true, row_total, x_bytes, keys);
+  };
+  if (m == 1) return go(std::integral_constant<int, 1>());
+  if (m == 2) return go(std::integral_constant<int, 2>());
+  if (m <= 4) return go(std::integral_constant<int, 4>());
+  return go(std::integral_constant<int, 8>());
+}
+
 }  // namespace
 
 int read_gemv_timeout_flag(int clear, unsigned *value) {
@@ -821,6 +900,30 @@ int read_gemv_timeout_flag(int clear, unsigned *value) {
 int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                      const DevInfo &dev, bool pdl) {
   return w.bits == 4 ? pick_mt<4>(x, m, w, y, s, dev, pdl) : pick_mt<8>(x, m, w, y, s, dev, pdl);
+}
+
+int launch_gemv_argmax(const float *x, int64_t m, const woq_weight &w, int64_t *idx, float *val,
+                       cudaStream_t s, const DevInfo &dev) {
+  unsigned long long *keys = reinterpret_cast<unsigned long long *>(idx);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(32, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, argmax_init_kernel, keys, static_cast<int>(m)) != cudaSuccess)
+    return WOQ_ECUDA;
+  count_launches(1);
+  const int rc = w.bits == 4 ? argmax_bulk<4>(x, m, w, keys, s, dev) : argmax_bulk<8>(x, m, w, keys, s, dev);
+  if (rc == 1) return WOQ_ESHAPE;
+  if (rc != WOQ_OK) return rc;
+  if (cudaLaunchKernelEx(&cfg, argmax_final_kernel, keys, val, static_cast<int>(m)) != cudaSuccess)
+    return WOQ_ECUDA;
+  count_launches(1);
+  return WOQ_OK;
 }
 
 }  // namespace woq

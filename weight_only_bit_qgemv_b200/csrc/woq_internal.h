@@ -36,6 +36,9 @@ bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType type, size_t esize, 
 // already validated. `pdl` launches with programmatic stream serialization.
 int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                      const DevInfo &dev, bool pdl);
+// qgemv_argmax: zero the keys in idx, the argmax GEMV, then keys -> (idx, val).
+int launch_gemv_argmax(const float *x, int64_t m, const woq_weight &w, int64_t *idx, float *val,
+                       cudaStream_t s, const DevInfo &dev);
 
 // Reads (and optionally clears) the GEMV kernels' record of bounded waits that gave up.
 int read_gemv_timeout_flag(int clear, unsigned *value);
