@@ -129,6 +129,19 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
                void *stream);
 
 /*
+ * qgemv_swiglu -- a fused gate|up projection and its SwiGLU: with W's rows interleaved
+ * (row 2i the gate row i, row 2i+1 the up row i; n = 2I), y[j, i] = silu(g) * u where
+ * g = (x . W_hat^T)[j, 2i], u = (x . W_hat^T)[j, 2i+1] and silu(g) = g / (1 + exp(-g)), the
+ * Qwen3-style MLP activation the decoder's feed-forward uses. The 2I projection outputs are
+ * never written. g and u are computed exactly as qgemv's CUDA-core form computes them.
+ *   x  device, [m, k] float32 row-major, 16-byte aligned, 1 <= m <= 64
+ *   w  host pointer to the weight descriptor; n even (rows interleaved as above)
+ *   y  device, [m, n/2] float32 row-major; fully overwritten
+ * Limits: k <= 8192. Errors: as qgemv, and WOQ_ESHAPE for an odd n.
+ */
+int qgemv_swiglu(const float *x, int64_t m, const woq_weight *w, float *y, void *stream);
+
+/*
  * qgemv_argmax -- greedy pick over a GEMV's outputs without writing them: for each activation
  * row i, idx[i] = the smallest j with y[i, j] = max over j of y[i, j], and val[i] = that
  * maximum, where y = x . W_hat^T is computed exactly as qgemv's CUDA-core form computes it.

@@ -27,6 +27,8 @@ from .woq_ref import (  # noqa: F401
     qgemm_ref,
     qgemm_bf16_ref,
     greedy_ref,
+    silu_ref,
+    swiglu_ref,
     qgemv_argmax_ref,
     bf16_round,
 )

@@ -183,6 +183,21 @@ def qgemm_bf16_ref(X: np.ndarray, packed: np.ndarray, scale_bits: np.ndarray, bi
     return matmul_ref(bf16_round(X), bf16_round(W_hat))
 
 
+def silu_ref(g: np.ndarray) -> np.ndarray:
+    """SiLU, g * sigmoid(g) = g / (1 + exp(-g)), in float64 (written as g * sigmoid for large
+    negative g, where exp(-g) overflows)."""
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return np.where(g >= 0, g / (1.0 + np.exp(-g)), g * np.exp(g) / (1.0 + np.exp(g)))
+
+
+def swiglu_ref(X: np.ndarray, packed: np.ndarray, scale_bits: np.ndarray, bits: int) -> np.ndarray:
+    """SwiGLU over a row-interleaved gate|up weight: Y = qgemv_ref(...), then
+    silu(Y[:, 0::2]) * Y[:, 1::2] in float64."""
+    Y = qgemv_ref(X, packed, scale_bits, bits)
+    return silu_ref(Y[:, 0::2]) * Y[:, 1::2]
+
+
 def greedy_ref(Y: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """Greedy decoding's pick over each row of outputs Y [M, N]: the first index of the
     row maximum, and that maximum ("MOSS Transcribe Diarize 0.9B", soniqo Russian guide,

@@ -68,6 +68,11 @@ def test_argument_checks_return_before_touching_a_device():
     assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, 3, None) == _lib.WOQ_EINVAL
     assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, -1, None) == _lib.WOQ_EINVAL
     assert L.qgemv_path(ok_ptr, 65, ctypes.byref(w), ok_ptr, _lib.WOQ_GEMV_SPLIT_TC, None) == _lib.WOQ_EINVAL
+    # qgemv_swiglu: 1 <= m <= 64, n even
+    assert L.qgemv_swiglu(ok_ptr, 0, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EINVAL
+    assert L.qgemv_swiglu(ok_ptr, 65, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EINVAL
+    odd = _w(n=63, packed=ok_ptr, scales=ok_ptr)
+    assert L.qgemv_swiglu(ok_ptr, 1, ctypes.byref(odd), ok_ptr, None) == _lib.WOQ_ESHAPE
     # qgemv_argmax: 1 <= m <= 8, k <= 8192, idx 8-byte aligned
     assert L.qgemv_argmax(ok_ptr, 0, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EINVAL
     assert L.qgemv_argmax(ok_ptr, 9, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EINVAL

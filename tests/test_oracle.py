@@ -380,3 +380,38 @@ def test_qgemv_argmax_ref_on_a_hand_built_weight():
     x[0, 0] = -2.0                                            # now -7 * -2 = 14 at j = 2
     idx, val = oracle.qgemv_argmax_ref(x, p, s, 4)
     assert idx.tolist() == [2] and val.tolist() == [14.0]
+
+
+# ---- SwiGLU (qgemv_swiglu reference) ----
+
+def test_silu_ref_invariants():
+    g = np.array([-700.0, -30.0, -2.5, -1e-3, 0.0, 1e-3, 0.7, 2.5, 30.0, 700.0])
+    s = oracle.silu_ref(g)
+    assert s[4] == 0.0
+    # silu(g) - silu(-g) = g (sigmoid(g) + sigmoid(-g) = 1)
+    assert np.allclose(s - oracle.silu_ref(-g), g, rtol=0, atol=1e-12 * np.maximum(1, np.abs(g)))
+    # limits: silu(g) -> g for large g, -> 0 for large negative g
+    assert s[-1] == 700.0 and s[-2] == pytest.approx(30.0, rel=1e-12)
+    assert abs(s[0]) < 1e-300 and abs(s[1]) < 30.0 * 1e-12
+    # slope 1/2 at 0: silu(h) / h -> 1/2
+    assert s[5] / 1e-3 == pytest.approx(0.5, rel=1e-3)
+    assert np.all(np.isfinite(s))
+
+
+def test_swiglu_ref_pairs_gate_and_up_rows():
+    # gate rows (even) and up rows (odd) built so that gate outputs are 0 or large
+    K = 32
+    W = np.zeros((4, K), dtype=np.float32)
+    W[0, :] = 0.0            # gate 0: output 0 -> silu 0
+    W[1, 0] = 7.0; W[1, 1] = 7.0   # up 0
+    W[2, 0] = 7.0; W[2, 1] = 7.0   # gate 1: output 7 * (x0 + x1)
+    W[3, 0] = -7.0; W[3, 1] = 7.0  # up 1: 7 * (x1 - x0)
+    q, s = oracle.quantise(W, 4)
+    p = oracle.pack(q, 4)
+    x = np.zeros((1, K), dtype=np.float32); x[0, 0] = 3.0; x[0, 1] = 5.0
+    y = oracle.swiglu_ref(x, p, s, 4)
+    assert y.shape == (1, 2)
+    assert y[0, 0] == 0.0
+    g, u = 7.0 * 8.0, 7.0 * 2.0
+    assert y[0, 1] == pytest.approx(oracle.silu_ref(np.array(g))[()] * u, rel=1e-15)
+    assert y[0, 1] == pytest.approx(g * u, rel=1e-20)  # sigmoid(56) is 1 to double precision

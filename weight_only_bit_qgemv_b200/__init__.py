@@ -34,6 +34,8 @@ __all__ = [
     "pack",
     "qgemv",
     "qgemv_argmax",
+    "qgemv_swiglu",
+    "interleave_rows",
     "qgemm",
     "qgemm_workspace_bytes",
     "device_status",
@@ -115,6 +117,26 @@ def qgemv(
     d = w.desc()
     rc = _lib.lib().qgemv_path(_ptr(x), m, ctypes.byref(d), _ptr(out), _GEMV_PATHS[path], _stream(stream))
     _lib.check(rc, "qgemv")
+    return out
+
+
+def interleave_rows(W_gate: torch.Tensor, W_up: torch.Tensor) -> torch.Tensor:
+    """[I, k] gate and up weights -> [2I, k] with row 2i = gate i, row 2i+1 = up i, the
+    layout qgemv_swiglu expects."""
+    if W_gate.shape != W_up.shape:
+        raise ValueError("gate and up weights must have the same shape")
+    return torch.stack([W_gate, W_up], dim=1).reshape(2 * W_gate.shape[0], W_gate.shape[1])
+
+
+def qgemv_swiglu(x: torch.Tensor, w: PackedWeight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[m, n/2] = silu(gate) * up over a row-interleaved gate|up weight (C ABI ``qgemv_swiglu``)."""
+    if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty(m, w.n // 2, dtype=torch.float32, device=x.device)
+    d = w.desc()
+    _lib.check(_lib.lib().qgemv_swiglu(_ptr(x), m, ctypes.byref(d), _ptr(out), _stream(stream)), "qgemv_swiglu")
     return out
 
 

@@ -30,6 +30,7 @@ EXPORTS = (
     "qpack",
     "qgemv",
     "qgemv_path",
+    "qgemv_swiglu",
     "qgemv_argmax",
     "qgemm_workspace_bytes",
     "qgemm",
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.qgemv.restype = ctypes.c_int
     L.qgemv_path.argtypes = [vp, c_i64, wp, vp, c_i32, vp]
     L.qgemv_path.restype = ctypes.c_int
+    L.qgemv_swiglu.argtypes = [vp, c_i64, wp, vp, vp]
+    L.qgemv_swiglu.restype = ctypes.c_int
     L.qgemv_argmax.argtypes = [vp, c_i64, wp, vp, vp, vp]
     L.qgemv_argmax.restype = ctypes.c_int
     L.qgemm_workspace_bytes.argtypes = [c_i64, wp, c_i32]

@@ -99,6 +99,19 @@ int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream
   return qgemv_path(x, m, w, y, WOQ_GEMV_AUTO, stream);
 }
 
+int qgemv_swiglu(const float *x, int64_t m, const woq_weight *w, float *y, void *stream) {
+  int rc = woq::check_weight(w);
+  if (rc != WOQ_OK) return rc;
+  if (!x || !y) return WOQ_EINVAL;
+  if (m < 1 || m > 64) return WOQ_EINVAL;
+  if (w->n % 2 != 0 || w->k > 8192) return WOQ_ESHAPE;
+  if (!woq::aligned(x, 16) || !woq::aligned(y, 4)) return WOQ_EALIGN;
+  DevInfo dev;
+  rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  return woq::launch_gemv_swiglu(x, m, *w, y, static_cast<cudaStream_t>(stream), dev);
+}
+
 int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, float *val,
                  void *stream) {
   int rc = woq::check_weight(w);

@@ -462,9 +462,15 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int row) {
   return (static_cast<unsigned long long>(o) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(row));
 }
 
-// AMAX = false: y[m, n] is written. AMAX = true: nothing is written to y; for each activation
-// row, the CTA's largest key over its outputs goes into keys[row] by a 64-bit atomicMax.
-template <int BITS, int MT, int RW, int NW, bool AMAX = false>
+// Epilogues. kEpiWrite: y[m, n] is written. kEpiArgmax: nothing is written to y; for each
+// activation row the CTA's largest key over its outputs goes into keys[row] by a 64-bit
+// atomicMax. kEpiSwiglu: rows 2i and 2i+1 are a gate and an up projection (RW even, so a
+// warp holds both); y[m, n/2] gets silu(gate) * up.
+constexpr int kEpiWrite = 0, kEpiArgmax = 1, kEpiSwiglu = 2;
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
 __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
                      const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n,
@@ -472,6 +478,8 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
                      unsigned long long *__restrict__ keys = nullptr) {
   constexpr int kBulkWarps = NW;
   constexpr int TR = kBulkWarps * RW;
+  constexpr bool AMAX = EPI == kEpiArgmax;
+  static_assert(EPI != kEpiSwiglu || RW % 2 == 0, "gate/up pairs need an even row count");
   extern __shared__ __align__(128) uint8_t smem[];
   BulkShared &sh = *reinterpret_cast<BulkShared *>(smem);
   float4 *xs4 = reinterpret_cast<float4 *>(smem + kBulkHeader);
@@ -609,8 +617,14 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
           if constexpr (AMAX) {
             const unsigned long long key = argmax_key(acc[r][mm], row0 + r);
             best = key > best ? key : best;
-          } else
+          } else if constexpr (EPI == kEpiSwiglu) {
+            // every lane holds every row's sum after the butterfly: the up row r + 1 is here
+            if (r % 2 == 0)
+              y[static_cast<size_t>(m0 + mm) * (n / 2) + (row0 + r) / 2] =
+                  silu(acc[r][mm]) * acc[r + 1 < RW ? r + 1 : r][mm];
+          } else {
             y[static_cast<size_t>(m0 + mm) * n + row0 + r] = acc[r][mm];
+          }
         }
   }
   if constexpr (AMAX) {
@@ -737,11 +751,11 @@ int pick_ru(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
 constexpr size_t kStageTarget = 20 * 1024;   // bytes per ring stage to aim for
 constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
 
-template <int BITS, int MT, int RW, int NW, bool AMAX = false>
+template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
 int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                   const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes,
                   unsigned long long *keys = nullptr) {
-  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW, AMAX>;
+  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW, EPI>;
   constexpr int kBulkThreads = bulk_threads(NW);
   constexpr int TR = NW * RW;
   const int64_t num_tiles = (w.n + TR - 1) / TR;
@@ -785,7 +799,7 @@ inline int bulk_rows_per_warp(int nw, int rw_max, size_t row_total) {
   return rw;
 }
 
-template <int BITS, int MT, int NW, bool AMAX = false>
+template <int BITS, int MT, int NW, int EPI = kEpiWrite>
 int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                    const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes,
                    unsigned long long *keys = nullptr) {
@@ -796,13 +810,13 @@ int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cud
   if (w.n < NW * rw) rw = 1;  // tiny n: one row per warp, all from global memory
   if constexpr (MT <= 2 && NW == 8) {
     if (rw == 4)
-      return launch_bulk_t<BITS, MT, 4, NW, AMAX>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
+      return launch_bulk_t<BITS, MT, 4, NW, EPI>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
   }
   if constexpr (NW == 8 || MT == 1) {
     if (rw >= 2)
-      return launch_bulk_t<BITS, MT, 2, NW, AMAX>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
+      return launch_bulk_t<BITS, MT, 2, NW, EPI>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
   }
-  return launch_bulk_t<BITS, MT, 1, NW, AMAX>(x, m, w, y, s, dev, pdl,
+  return launch_bulk_t<BITS, MT, 1, NW, EPI>(x, m, w, y, s, dev, pdl,
                                               (static_cast<size_t>(NW) * row_total + 127) & ~size_t(127),
                                               x_bytes, keys);
 }
@@ -869,6 +883,32 @@ __global__ void __launch_bounds__(32) argmax_final_kernel(unsigned long long *ke
       static_cast<long long>(0xFFFFFFFFu - static_cast<uint32_t>(key & 0xFFFFFFFFull));
 }
 
+// qgemv_swiglu: the bulk GEMV with two rows (gate, up) per warp.
+template <int BITS>
+int swiglu_bulk(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                const DevInfo &dev) {
+  const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
+  auto go = [&](auto mt_tag, auto nw_tag) -> int {
+    constexpr int MT = decltype(mt_tag)::value;
+    constexpr int NW = decltype(nw_tag)::value;
+    const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
+    const size_t stage_bytes = (static_cast<size_t>(NW) * 2 * row_total + 127) & ~size_t(127);
+    if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return WOQ_ESHAPE;
+    return launch_bulk_t<BITS, MT, 2, NW, kEpiSwiglu>(x, m, w, y, s, dev, true, stage_bytes, x_bytes);
+  };
+  using I1 = std::integral_constant<int, 1>;
+  using I8 = std::integral_constant<int, 8>;
+  using I16 = std::integral_constant<int, 16>;
+  if (m == 1) {
+    // as qgemv: 16 warps while each CTA gets at most two tiles
+    if (w.n / 32 <= 2 * static_cast<int64_t>(dev.sm_count)) return go(I1(), I16());
+    return go(I1(), I8());
+  }
+  if (m == 2) return go(std::integral_constant<int, 2>(), I8());
+  if (m <= 4) return go(std::integral_constant<int, 4>(), I8());
+  return go(I8(), I8());
+}
+
 template <int BITS>
 int argmax_bulk(const float *x, int64_t m, const woq_weight &w, unsigned long long *keys,
                 cudaStream_t s, const DevInfo &dev) {
@@ -876,7 +916,7 @@ int argmax_bulk(const float *x, int64_t m, const woq_weight &w, unsigned long lo
   auto go = [&](auto mt_tag) -> int {
     constexpr int MT = decltype(mt_tag)::value;
     const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
-    return launch_bulk_nw<BITS, MT, 8, true>(x, m, w, nullptr, s, dev, true, row_total, x_bytes, keys);
+    return launch_bulk_nw<BITS, MT, 8, kEpiArgmax>(x, m, w, nullptr, s, dev, true, row_total, x_bytes, keys);
   };
   if (m == 1) return go(std::integral_constant<int, 1>());
   if (m == 2) return go(std::integral_constant<int, 2>());
@@ -900,6 +940,11 @@ int read_gemv_timeout_flag(int clear, unsigned *value) {
 int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                      const DevInfo &dev, bool pdl) {
   return w.bits == 4 ? pick_mt<4>(x, m, w, y, s, dev, pdl) : pick_mt<8>(x, m, w, y, s, dev, pdl);
+}
+
+int launch_gemv_swiglu(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                       const DevInfo &dev) {
+  return w.bits == 4 ? swiglu_bulk<4>(x, m, w, y, s, dev) : swiglu_bulk<8>(x, m, w, y, s, dev);
 }
 
 int launch_gemv_argmax(const float *x, int64_t m, const woq_weight &w, int64_t *idx, float *val,
