@@ -57,9 +57,11 @@ extern "C" {
 #define WOQ_EWORKSPACE -8  /* qgemm: workspace null or smaller than qgemm_workspace_bytes     */
 
 /* qgemm paths. */
-#define WOQ_PATH_AUTO     0  /* BF16_TC when m >= 128 (see qgemm), FP32 otherwise          */
+#define WOQ_PATH_AUTO     0  /* by m: BF16_TC, SPLIT_TC or FP32 (see qgemm)                */
 #define WOQ_PATH_FP32     1  /* FP32 products and accumulation (CUDA cores), exact codes      */
 #define WOQ_PATH_BF16_TC  2  /* tcgen05 tensor cores on bf16(X) and bf16(scale*code)          */
+#define WOQ_PATH_SPLIT_TC 3  /* tcgen05 tensor cores, FP32-accurate: X and scale*code each as  */
+                             /* bf16 hi + bf16 lo, all four products accumulated in FP32      */
 
 /*
  * One packed weight [n, k] in device memory.
@@ -171,8 +173,16 @@ size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path);
  *   path WOQ_PATH_BF16_TC: X is rounded to bf16 into the workspace, each weight tile is
  *        dequantised once into shared memory as bf16(scale*code) and multiplied on the
  *        tcgen05 tensor cores with FP32 accumulation in tensor memory.
+ *   path WOQ_PATH_SPLIT_TC: FP32 accuracy on the tcgen05 tensor cores. Each x value is
+ *        split into hi = bf16(x) and lo = bf16(x - hi), and each dequantised weight
+ *        v = scale*code (exact in FP32) into hi = bf16(v) and lo = bf16(v - hi); the tiles
+ *        hold 64 activation rows, and one MMA per operand half multiplies the weight tile
+ *        against both X halves, so all four products land in the FP32 accumulator. For
+ *        int4, v_hi + v_lo == v exactly; x (and an int8 v) keeps 16 significand bits.
+ *        Four times the tensor-core work of BF16_TC; meant for small batches (m <= 64)
+ *        whose FP32 CUDA-core cost grows with m.
  *   path WOQ_PATH_FP32: the same FP32 arithmetic as qgemv, for any m.
- *   path WOQ_PATH_AUTO: BF16_TC if m >= 128, else FP32.
+ *   path WOQ_PATH_AUTO: BF16_TC if m >= 128, SPLIT_TC if 24 <= m < 128, else FP32.
  *   X  device, [m, k] float32 row-major, 16-byte aligned
  *   Y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
  *   workspace  device, 256-byte aligned, at least qgemm_workspace_bytes(m, w, path) bytes

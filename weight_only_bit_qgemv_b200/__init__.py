@@ -25,6 +25,7 @@ from ._lib import (  # noqa: F401
     WOQ_PATH_AUTO,
     WOQ_PATH_BF16_TC,
     WOQ_PATH_FP32,
+    WOQ_PATH_SPLIT_TC,
     WoqError,
 )
 
@@ -43,7 +44,12 @@ __all__ = [
     "WoqError",
 ]
 
-_PATHS = {"auto": WOQ_PATH_AUTO, "fp32": WOQ_PATH_FP32, "bf16_tc": WOQ_PATH_BF16_TC}
+_PATHS = {
+    "auto": WOQ_PATH_AUTO,
+    "fp32": WOQ_PATH_FP32,
+    "bf16_tc": WOQ_PATH_BF16_TC,
+    "split_tc": WOQ_PATH_SPLIT_TC,
+}
 _GEMV_PATHS = {"auto": WOQ_GEMV_AUTO, "cuda_core": WOQ_GEMV_CUDA_CORE, "split_tc": WOQ_GEMV_SPLIT_TC}
 
 
@@ -167,7 +173,7 @@ def qgemm(
     workspace: torch.Tensor | None = None,
     stream=None,
 ) -> torch.Tensor:
-    """Y[m, n] = X[m, k] . W_hat^T (C ABI ``qgemm``); path in {"auto", "fp32", "bf16_tc"}."""
+    """Y[m, n] = X[m, k] . W_hat^T (C ABI ``qgemm``); path in {"auto", "fp32", "bf16_tc", "split_tc"}."""
     if X.dtype != torch.float32 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
         raise ValueError("X must be a contiguous 2-D float32 CUDA tensor")
     m = X.shape[0]

@@ -21,6 +21,7 @@ WOQ_EWORKSPACE = -8
 WOQ_PATH_AUTO = 0
 WOQ_PATH_FP32 = 1
 WOQ_PATH_BF16_TC = 2
+WOQ_PATH_SPLIT_TC = 3
 WOQ_GEMV_AUTO = 0
 WOQ_GEMV_CUDA_CORE = 1
 WOQ_GEMV_SPLIT_TC = 2

@@ -133,16 +133,29 @@ static int plan_sm_count() {
   return woq::current_device(&dev) == WOQ_OK ? dev.sm_count : 0;
 }
 
+// qgemm's automatic choice: the bf16 tensor-core GEMM for prefill-sized m, the FP32-accurate
+// split tensor-core GEMM for batched decode from kSplitMinM rows on (measured on B200 over
+// the decoder projections: faster than the CUDA-core kernel from there on), and the CUDA-core
+// kernel below that.
+constexpr int64_t kSplitMinM = 24;
+
 static int resolve_path(int32_t path, int64_t m) {
-  if (path == WOQ_PATH_AUTO) return m >= 128 ? WOQ_PATH_BF16_TC : WOQ_PATH_FP32;
+  if (path == WOQ_PATH_AUTO)
+    return m >= 128 ? WOQ_PATH_BF16_TC : m >= kSplitMinM ? WOQ_PATH_SPLIT_TC : WOQ_PATH_FP32;
   return path;
+}
+
+static bool known_path(int32_t path) {
+  return path == WOQ_PATH_AUTO || path == WOQ_PATH_FP32 || path == WOQ_PATH_BF16_TC ||
+         path == WOQ_PATH_SPLIT_TC;
 }
 
 size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path) {
   if (woq::check_weight(w) != WOQ_OK || m < 1) return 0;
-  if (path != WOQ_PATH_AUTO && path != WOQ_PATH_FP32 && path != WOQ_PATH_BF16_TC) return 0;
-  if (resolve_path(path, m) != WOQ_PATH_BF16_TC) return 0;
-  return woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX).total;
+  if (!known_path(path)) return 0;
+  const int p = resolve_path(path, m);
+  if (p == WOQ_PATH_FP32) return 0;
+  return woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX, p == WOQ_PATH_SPLIT_TC).total;
 }
 
 int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path,
@@ -151,13 +164,13 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
   if (rc != WOQ_OK) return rc;
   if (!X || !Y) return WOQ_EINVAL;
   if (m < 1 || m > INT32_MAX) return WOQ_EINVAL;
-  if (path != WOQ_PATH_AUTO && path != WOQ_PATH_FP32 && path != WOQ_PATH_BF16_TC) return WOQ_EINVAL;
+  if (!known_path(path)) return WOQ_EINVAL;
   if (!woq::aligned(X, 16) || !woq::aligned(Y, 16)) return WOQ_EALIGN;
   const int p = resolve_path(path, m);
   if (p == WOQ_PATH_FP32 && w->k > 32768) return WOQ_ESHAPE;
   woq::GemmPlan plan;
-  if (p == WOQ_PATH_BF16_TC) {
-    plan = woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX);
+  if (p != WOQ_PATH_FP32) {
+    plan = woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX, p == WOQ_PATH_SPLIT_TC);
     if (!workspace || workspace_bytes < plan.total) return WOQ_EWORKSPACE;
     if (!woq::aligned(workspace, 256)) return WOQ_EALIGN;
   }

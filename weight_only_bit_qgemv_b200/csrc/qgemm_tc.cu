@@ -43,13 +43,14 @@ constexpr int kMaxSL = 8;           // load stages (X tile + raw code tile)
 constexpr int kMaxSB = 4;           // dequantised weight tiles (ring), at most
 // Weight-tile ring depth: 4 for 128-row tiles (the dequantisers then run two stages ahead
 // of the MMAs instead of waiting on each stage's completion), 2 for 256-row tiles.
-__host__ __device__ constexpr int sb_for(int bn) { return bn == 128 ? 4 : 2; }
+__host__ __device__ constexpr int sb_for(int bn, bool split = false) {
+  return split ? 3 : bn == 128 ? 4 : 2;
+}
 constexpr int kTmaScaleCols = 128;  // scale tile copied by TMA when K/32 <= this (and % 8 == 0)
 constexpr int kDequantWarps = 16;  // four per scheduler: each warp's chain is latency-bound
 constexpr int kDequantThreads = kDequantWarps * 32;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = (2 + kDequantWarps + kEpiWarps) * 32;  // 704
-constexpr int kABytes = BM * BK * 2;                            // 16 KB
 constexpr long long kDrainLimit = 1LL << 31;                    // cycles (~1 s)
 constexpr long long kDefaultWaitLimit = 1LL << 32;              // cycles (~2 s)
 constexpr int kSmemMax = 227 * 1024;
@@ -85,13 +86,13 @@ struct Shared {
 struct Layout {
   int a, b, raw, sc, bar, total;
 };
-__host__ __device__ inline Layout make_layout(int bits, int bn, int mh, int sl, int sc_bytes,
-                                              int sc_bufs) {
+__host__ __device__ inline Layout make_layout(int bits, int bn, int x_stage, int b_slot, int sb,
+                                              int sl, int sc_bytes, int sc_bufs) {
   Layout L;
   const int raw_bytes = bn * BK * bits / 8;
   L.a = 0;
-  L.b = L.a + sl * mh * kABytes;
-  L.raw = L.b + sb_for(bn) * bn * BK * 2;
+  L.b = L.a + sl * x_stage;
+  L.raw = L.b + sb * b_slot;
   L.sc = L.raw + sl * raw_bytes;
   L.bar = (L.sc + sc_bufs * sc_bytes + 127) & ~127;
   L.total = L.bar + static_cast<int>(sizeof(Shared)) + 1024;  // + base alignment slack
@@ -159,7 +160,59 @@ __device__ __forceinline__ uint4 dequant_int8_words(uint32_t w0, uint32_t w1, fl
   return out;
 }
 
-template <int BITS, int BN, int MH>
+// Split forms for the FP32-accurate tensor-core path: the exact FP32 value v = s*q as
+// bf16 hi = RNE(v) plus bf16 lo = RNE(v - hi). For int4, v has at most 15 significant bits,
+// so hi + lo == v exactly; for int8 the remainder below lo is under 2^-16 of |v|.
+__device__ __forceinline__ void split_pack(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+__device__ __forceinline__ void dequant_int4_word_split(uint32_t w, const float (&sj)[4], uint4 &hi,
+                                                        uint4 &lo) {
+  const uint32_t hw = w >> 16;
+  float2 v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t mask = 0xFu << (4 * j);
+    const uint32_t magic = 0x4B000000u | (0x8u << (4 * j));
+    const float bias = 8388608.0f + 8.0f * static_cast<float>(1u << (4 * j));
+    v[j] = __fadd2_rn(make_float2(__uint_as_float((w & mask) ^ magic), __uint_as_float((hw & mask) ^ magic)),
+                      make_float2(-bias, -bias));
+    v[j] = __fmul2_rn(v[j], make_float2(sj[j], sj[j]));
+  }
+  split_pack(v[0].x, v[1].x, hi.x, lo.x);
+  split_pack(v[2].x, v[3].x, hi.y, lo.y);
+  split_pack(v[0].y, v[1].y, hi.z, lo.z);
+  split_pack(v[2].y, v[3].y, hi.w, lo.w);
+}
+
+__device__ __forceinline__ void dequant_int8_words_split(uint32_t w0, uint32_t w1, float s, uint4 &hi,
+                                                         uint4 &lo) {
+  const float bias = 8388608.0f + 128.0f;
+  const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;
+  float2 p[4];
+  p[0] = make_float2(__uint_as_float(__byte_perm(u0, 0x4B000000u, 0x7540)),
+                     __uint_as_float(__byte_perm(u0, 0x4B000000u, 0x7541)));
+  p[1] = make_float2(__uint_as_float(__byte_perm(u0, 0x4B000000u, 0x7542)),
+                     __uint_as_float(__byte_perm(u0, 0x4B000000u, 0x7543)));
+  p[2] = make_float2(__uint_as_float(__byte_perm(u1, 0x4B000000u, 0x7540)),
+                     __uint_as_float(__byte_perm(u1, 0x4B000000u, 0x7541)));
+  p[3] = make_float2(__uint_as_float(__byte_perm(u1, 0x4B000000u, 0x7542)),
+                     __uint_as_float(__byte_perm(u1, 0x4B000000u, 0x7543)));
+  uint32_t *h = reinterpret_cast<uint32_t *>(&hi), *l = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 v = __fadd2_rn(p[i], make_float2(-bias, -bias));
+    v = __fmul2_rn(v, make_float2(s, s));
+    split_pack(v.x, v.y, h[i], l[i]);
+  }
+}
+
+template <int BITS, int BN, int MH, bool SPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s, const uint16_t *__restrict__ scales,
@@ -168,21 +221,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     long long stuck_wait) {
   constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
   constexpr int kRawBytes = BN * kRawRow;
-  constexpr int kBBytes = BN * BK * 2;
-  constexpr int kSB = sb_for(BN);              // weight-tile ring depth
-  constexpr int TM = BM * MH;                   // output rows (activation rows) per tile
-  constexpr int kAStage = MH * kABytes;         // X bytes per load stage
+  // SPLIT (FP32-accurate form): each X tile holds 64 activation rows as bf16 hi then bf16 lo
+  // (128 rows), each weight slot holds the bf16 hi and lo tiles of the dequantised weights,
+  // and per K-step two M=128, N=128 MMAs (A = weight hi, then weight lo; B = the X tile)
+  // accumulate all four products; the epilogue adds the hi and lo column halves.
+  static_assert(!SPLIT || (MH == 1 && BN == BM), "the split form uses 128-row weight tiles");
+  constexpr bool kSwap = MH == 2 || SPLIT;       // A = weight tile, B = X tile
+  constexpr int kBBytes1 = BN * BK * 2;          // one dequantised weight tile
+  constexpr int kBBytes = (SPLIT ? 2 : 1) * kBBytes1;  // one weight ring slot
+  constexpr int kSB = sb_for(BN, SPLIT);         // weight-tile ring depth
+  constexpr int TM = SPLIT ? 64 : BM * MH;       // output rows (activation rows) per tile
+  constexpr int kXRows = SPLIT ? 128 : TM;       // X tile rows per stage
+  constexpr int kAStage = kXRows * BK * 2;       // X bytes per load stage
   // MH = 1: the MMA's A is the X tile and B the weight tile; the accumulator holds
   // [128 activation rows x BN]. MH = 2: the roles swap, A = the 128-row weight tile and
   // B = the 256-row X tile, so one M=128, N=256 MMA per K-step covers the whole tile (long
   // MMAs keep the tensor pipe fed between stages); the accumulator holds [BN = 128 weight
   // rows x 256 activation rows].
   static_assert(MH == 1 || BN == BM, "swapped tiles need 128 weight rows");
-  constexpr int kAccCols = MH == 2 ? TM : BN;   // accumulator columns per set
-  constexpr uint32_t kTmemCols = 2 * kAccCols;  // two accumulator sets
+  constexpr int kAccCols = kSwap ? kXRows : BN;  // accumulator columns per set (= MMA N)
+  constexpr uint32_t kTmemCols = 2 * kAccCols;   // two accumulator sets
   static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
-  constexpr uint32_t kIdesc = idesc_for(MH == 2 ? TM : BN);
-  const Layout L = make_layout(BITS, BN, MH, sl_stages, sc_bytes, sc_bufs);
+  constexpr uint32_t kIdesc = idesc_for(kAccCols);
+  const Layout L = make_layout(BITS, BN, kAStage, kBBytes, kSB, sl_stages, sc_bytes, sc_bufs);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -280,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::pdl_wait();
             waited = true;
           }
-          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.wfull[s], ks * BK, mb * TM);
+          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.wfull[s], ks * BK, mb * kXRows);
           if (++s == SL) {
             s = 0;
             ph ^= 1;
@@ -318,16 +379,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          // start-address field counts 16-byte units; K=16 bf16 = 32 bytes = 2 units; the
-          // second 128-row half of the X tile starts kABytes further on
+          // start-address field counts 16-byte units; K=16 bf16 = 32 bytes = 2 units; in the
+          // split form the lo half of the weight tile starts kBBytes1 further on
           const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kAStage >> 4));
           const uint64_t bd = bdesc0 + static_cast<uint64_t>(bs * (kBBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            if constexpr (MH == 2)
-              ptx::tc_mma_f16(d, bd + 2 * kk, ad + 2 * kk, kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
-            else
-              ptx::tc_mma_f16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (ks != ks0 || kk != 0) ? 1u : 0u);
+            const uint32_t acc = (ks != ks0 || kk != 0) ? 1u : 0u;
+            if constexpr (SPLIT) {
+              ptx::tc_mma_f16(d, bd + 2 * kk, ad + 2 * kk, kIdesc, acc);
+              ptx::tc_mma_f16(d, bd + (kBBytes1 >> 4) + 2 * kk, ad + 2 * kk, kIdesc, 1u);
+            } else if constexpr (MH == 2) {
+              ptx::tc_mma_f16(d, bd + 2 * kk, ad + 2 * kk, kIdesc, acc);
+            } else {
+              ptx::tc_mma_f16(d, ad + 2 * kk, bd + 2 * kk, kIdesc, acc);
+            }
           }
           mma_issued = true;
           ptx::tc_commit(&sh.lempty[s]);
@@ -405,7 +471,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < CH; ++i) {
             const int chunk = part * CH + i;
-            *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) = dequant_int4_word(ws[i], sj);
+            if constexpr (SPLIT) {
+              uint4 hi, lo;
+              dequant_int4_word_split(ws[i], sj, hi, lo);
+              *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) = hi;
+              *reinterpret_cast<uint4 *>(brow + kBBytes1 + ((chunk ^ sw) << 4)) = lo;
+            } else {
+              *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) = dequant_int4_word(ws[i], sj);
+            }
           }
         } else {
           uint32_t ws[2 * CH];  // two words = 8 codes = one chunk
@@ -417,8 +490,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < CH; ++i) {
             const int chunk = part * CH + i;
-            *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) =
-                dequant_int8_words(ws[2 * i], ws[2 * i + 1], s0);
+            if constexpr (SPLIT) {
+              uint4 hi, lo;
+              dequant_int8_words_split(ws[2 * i], ws[2 * i + 1], s0, hi, lo);
+              *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) = hi;
+              *reinterpret_cast<uint4 *>(brow + kBBytes1 + ((chunk ^ sw) << 4)) = lo;
+            } else {
+              *reinterpret_cast<uint4 *>(brow + ((chunk ^ sw) << 4)) =
+                  dequant_int8_words(ws[2 * i], ws[2 * i + 1], s0);
+            }
           }
         }
         // Each lane makes its writes visible to the async proxy (the tensor core), the warp
@@ -470,58 +550,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int n0 = nb * BN;
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
-      // 16-column chunks, software-pipelined: the next chunk's TMEM load is in flight while
-      // this one is stored (two register buffers, each waited for before use).
-      const int ncols = MH == 2 ? min(TM, M - mb * TM) : BN;
-      const int nchunks = (ncols + 15) / 16;
-      auto store_chunk = [&](const uint32_t (&r)[16], int c) {
-        const int c0 = 16 * c;
-        if constexpr (MH == 2) {
-          // TMEM lane = weight row n, column = activation row m: for each column the warp's
-          // 32 lanes store 32 consecutive floats of one Y row. The row pointer advances by
-          // N per column; full chunks skip the row check.
-          const int n = n0 + q * 32 + lane;
-          const int mrem = M - (mb * TM + c0);
+      if constexpr (SPLIT) {
+        // TMEM lane = weight row n; column t holds the token's hi part, column 64 + t its lo
+        // part: Y[m][n] is their sum. Each 16-column chunk loads both halves.
+        const int n = n0 + q * 32 + lane;
+        const int ncols = min(TM, M - mb * TM);
+        for (int c0 = 0; c0 < ncols; c0 += 16) {  // warp-uniform trip count
+          uint32_t ra[16], rb[16];
+          ptx::tmem_ld_32x32b_x16(tb + c0, ra);
+          ptx::tmem_ld_32x32b_x16(tb + TM + c0, rb);
+          ptx::tmem_ld_wait(ra);
+          ptx::tmem_ld_wait(rb);
+          const int mrem = ncols - c0;
           float *p = out + static_cast<size_t>(mb * TM + c0) * N + n;
           if (n < N) {
-            if (mrem >= 16) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j, p += N) *p = __uint_as_float(r[j]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 16; ++j, p += N)
-                if (j < mrem) *p = __uint_as_float(r[j]);
-            }
-          }
-        } else {
-          const int grow = mb * TM + q * 32 + lane;
-          if (grow < M) {
-            float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
-            if (vec && n0 + c0 + 16 <= N) {
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                reinterpret_cast<float4 *>(yr)[v] =
-                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-            } else {
-#pragma unroll
-              for (int v = 0; v < 16; ++v)
-                if (n0 + c0 + v < N) yr[v] = __uint_as_float(r[v]);
-            }
+            for (int j = 0; j < 16; ++j, p += N)
+              if (j < mrem) *p = __uint_as_float(ra[j]) + __uint_as_float(rb[j]);
           }
         }
-      };
-      uint32_t ra[16], rb[16];
-      ptx::tmem_ld_32x32b_x16(tb, ra);
-      ptx::tmem_ld_wait(ra);
-      for (int c = 0; c < nchunks; c += 2) {  // trip counts are warp-uniform
-        if (c + 1 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 1), rb);
-        store_chunk(ra, c);
-        if (c + 1 < nchunks) {
-          ptx::tmem_ld_wait(rb);
-          if (c + 2 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 2), ra);
-          store_chunk(rb, c + 1);
-          if (c + 2 < nchunks) ptx::tmem_ld_wait(ra);
+      } else {
+        // 16-column chunks, software-pipelined: the next chunk's TMEM load is in flight while
+        // this one is stored (two register buffers, each waited for before use).
+        const int ncols = MH == 2 ? min(TM, M - mb * TM) : BN;
+        const int nchunks = (ncols + 15) / 16;
+        auto store_chunk = [&](const uint32_t (&r)[16], int c) {
+          const int c0 = 16 * c;
+          if constexpr (MH == 2) {
+            // TMEM lane = weight row n, column = activation row m: for each column the warp's
+            // 32 lanes store 32 consecutive floats of one Y row. The row pointer advances by
+            // N per column; full chunks skip the row check.
+            const int n = n0 + q * 32 + lane;
+            const int mrem = M - (mb * TM + c0);
+            float *p = out + static_cast<size_t>(mb * TM + c0) * N + n;
+            if (n < N) {
+              if (mrem >= 16) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j, p += N) *p = __uint_as_float(r[j]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j, p += N)
+                  if (j < mrem) *p = __uint_as_float(r[j]);
+              }
+            }
+          } else {
+            const int grow = mb * TM + q * 32 + lane;
+            if (grow < M) {
+              float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
+              if (vec && n0 + c0 + 16 <= N) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  reinterpret_cast<float4 *>(yr)[v] =
+                      make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                  __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+              } else {
+#pragma unroll
+                for (int v = 0; v < 16; ++v)
+                  if (n0 + c0 + v < N) yr[v] = __uint_as_float(r[v]);
+              }
+            }
+          }
+        };
+        uint32_t ra[16], rb[16];
+        ptx::tmem_ld_32x32b_x16(tb, ra);
+        ptx::tmem_ld_wait(ra);
+        for (int c = 0; c < nchunks; c += 2) {  // trip counts are warp-uniform
+          if (c + 1 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 1), rb);
+          store_chunk(ra, c);
+          if (c + 1 < nchunks) {
+            ptx::tmem_ld_wait(rb);
+            if (c + 2 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 2), ra);
+            store_chunk(rb, c + 1);
+            if (c + 2 < nchunks) ptx::tmem_ld_wait(ra);
+          }
         }
       }
       ptx::tc_fence_before();
@@ -577,6 +678,27 @@ __global__ void __launch_bounds__(256) x_to_bf16_kernel(const float4 *__restrict
   }
 }
 
+// X fp32 [m, k] -> per 64-token tile t, workspace rows 128t .. 128t+63 = bf16 hi = RNE(x)
+// and rows 128t+64 .. 128t+127 = bf16 lo = RNE(x - hi); 8 elements per thread.
+__global__ void __launch_bounds__(256) x_split_kernel(const float4 *__restrict__ x,
+                                                      uint4 *__restrict__ xs, int k8, size_t n8) {
+  ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t row = i / k8, col = i - row * k8;
+    const float4 a = x[2 * i], b = x[2 * i + 1];
+    uint4 h, l;
+    split_pack(a.x, a.y, h.x, l.x);
+    split_pack(a.z, a.w, h.y, l.y);
+    split_pack(b.x, b.y, h.z, l.z);
+    split_pack(b.z, b.w, h.w, l.w);
+    const size_t base = (row / 64) * 128 + (row % 64);
+    xs[base * k8 + col] = h;
+    xs[(base + 64) * k8 + col] = l;
+  }
+}
+
 // Y = sum over splits of the FP32 partials, in split order (deterministic); 4 per thread.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4 *__restrict__ part,
                                                             float4 *__restrict__ y, size_t n4,
@@ -618,11 +740,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int BITS, int BN, int MH>
+template <int BITS, int BN, int MH, bool SPLIT = false>
 int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
               const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
-  auto kern = qgemm_tc_kernel<BITS, BN, MH>;
-  constexpr int TM = BM * MH;
+  auto kern = qgemm_tc_kernel<BITS, BN, MH, SPLIT>;
+  constexpr int TM = SPLIT ? 64 : BM * MH;      // activation rows per output tile
+  constexpr int kXRows = SPLIT ? 128 : TM;      // X workspace rows per output tile
+  constexpr int kAStage = kXRows * BK * 2;
+  constexpr int kBSlot = (SPLIT ? 2 : 1) * BN * BK * 2;
+  constexpr int kSB = sb_for(BN, SPLIT);
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
@@ -637,19 +763,24 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   const int64_t spr = w.k / 32;
   const bool sc_tma = spr % 8 == 0 && spr <= kTmaScaleCols;
   const int sc_bytes = sc_tma ? static_cast<int>((BN * spr * 2 + 127) & ~int64_t(127)) : 0;
-  const int stage = MH * kABytes + BN * BK * BITS / 8;
+  const int stage = kAStage + BN * BK * BITS / 8;
   auto stages_for = [&](int bufs) {
-    return std::min(kMaxSL, (kSmemMax - make_layout(BITS, BN, MH, 0, sc_bytes, bufs).total) / stage);
+    return std::min(kMaxSL,
+                    (kSmemMax - make_layout(BITS, BN, kAStage, kBSlot, kSB, 0, sc_bytes, bufs).total) /
+                        stage);
   };
   int sc_bufs = sc_tma ? 2 : 1;
   if (sc_tma && stages_for(2) < 4) sc_bufs = 1;
   const int sl = stages_for(sc_bufs);
   if (sl < 2) return WOQ_ESHAPE;
-  const int smem = make_layout(BITS, BN, MH, sl, sc_bytes, sc_bufs).total;
+  const int smem = make_layout(BITS, BN, kAStage, kBSlot, kSB, sl, sc_bytes, sc_bufs).total;
 
+  // The split form's workspace holds 128 rows (hi, then lo) per 64-token tile.
+  const int64_t num_m = (m + TM - 1) / TM;
+  const int64_t x_rows = SPLIT ? num_m * kXRows : m;
   CUtensorMap tm_x, tm_w, tm_s;
-  if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK, TM,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, x_rows, BK,
+                          kXRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return WOQ_ECUDA;
   if (!make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
                 BK * BITS / 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -666,7 +797,7 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
 
-  // 1) X -> bf16 into the workspace.
+  // 1) X -> bf16 (or bf16 hi + lo) into the workspace.
   const size_t n8 = static_cast<size_t>(m) * w.k / 8;
   {
     cudaLaunchConfig_t cfg = {};
@@ -677,15 +808,20 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, x_to_bf16_kernel, reinterpret_cast<const float4 *>(X),
-                           reinterpret_cast<uint4 *>(workspace), n8) != cudaSuccess)
-      return WOQ_ECUDA;
+    cudaError_t e;
+    if constexpr (SPLIT)
+      e = cudaLaunchKernelEx(&cfg, x_split_kernel, reinterpret_cast<const float4 *>(X),
+                             reinterpret_cast<uint4 *>(workspace), static_cast<int>(w.k / 8), n8);
+    else
+      e = cudaLaunchKernelEx(&cfg, x_to_bf16_kernel, reinterpret_cast<const float4 *>(X),
+                             reinterpret_cast<uint4 *>(workspace), n8);
+    if (e != cudaSuccess) return WOQ_ECUDA;
     count_launches(1);
   }
   // 2) the persistent GEMM: one CTA per SM (or per work unit, if fewer).
   float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + plan.xb);
   {
-    const int64_t tiles = ((m + TM - 1) / TM) * ((w.n + BN - 1) / BN) * plan.splits;
+    const int64_t tiles = num_m * ((w.n + BN - 1) / BN) * plan.splits;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(tiles, dev.sm_count)), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -738,17 +874,26 @@ bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType type, size_t esize, 
 }
 
 
-GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget) {
+GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget,
+                      bool split) {
   auto align = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };
   GemmPlan p;
-  p.xb = align(static_cast<size_t>(m) * static_cast<size_t>(k) * 2);
+  p.split = split;
   const int64_t num_k = (k + BK - 1) / BK;
-  // Past one 128-row M tile, 256 x 128 tiles (two M halves sharing each dequantised weight
-  // tile) halve the dequantisation per FLOP. Otherwise 128 x 256 tiles, which do twice the
-  // work per MMA instruction, when N allows.
-  p.mh = m > 128 ? 2 : 1;
-  p.bn = p.mh == 1 && n >= 256 ? 256 : 128;
-  const int64_t mt = (m + 128 * p.mh - 1) / (128 * p.mh);
+  int64_t mt;
+  if (split) {
+    // 64-token tiles; the workspace holds 128 rows (hi, then lo) per tile.
+    mt = (m + 63) / 64;
+    p.xb = align(static_cast<size_t>(mt) * 128 * static_cast<size_t>(k) * 2);
+  } else {
+    // Past one 128-row M tile, 256 x 128 tiles (two M halves sharing each dequantised
+    // weight tile) halve the dequantisation per FLOP. Otherwise 128 x 256 tiles, which do
+    // twice the work per MMA instruction, when N allows.
+    p.xb = align(static_cast<size_t>(m) * static_cast<size_t>(k) * 2);
+    p.mh = m > 128 ? 2 : 1;
+    p.bn = p.mh == 1 && n >= 256 ? 256 : 128;
+    mt = (m + 128 * p.mh - 1) / (128 * p.mh);
+  }
   int64_t tiles = mt * ((n + p.bn - 1) / p.bn);
   // Split K until the work units cover the SMs, keeping >= 4 K-stages per split; the splits
   // need FP32 partials in the workspace and a vectorisable Y (n % 4 == 0).
@@ -767,6 +912,9 @@ GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budg
 
 int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
                    const GemmPlan &plan, cudaStream_t s, const DevInfo &dev) {
+  if (plan.split)
+    return w.bits == 4 ? launch_tc<4, 128, 1, true>(X, m, w, Y, workspace, plan, s, dev)
+                       : launch_tc<8, 128, 1, true>(X, m, w, Y, workspace, plan, s, dev);
   if (w.bits == 4) {
     if (plan.mh == 2) return launch_tc<4, 128, 2>(X, m, w, Y, workspace, plan, s, dev);
     return plan.bn == 256 ? launch_tc<4, 256, 1>(X, m, w, Y, workspace, plan, s, dev)

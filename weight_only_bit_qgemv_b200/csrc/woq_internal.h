@@ -60,12 +60,15 @@ struct GemmPlan {
   int bn = 128;   // output columns per tile
   int mh = 1;     // 128-row M halves per tile (2: both share each dequantised weight tile)
   int splits = 1;
+  bool split = false;  // FP32-accurate form: X and W each as bf16 hi + bf16 lo
   size_t xb = 0, part = 0, total = 0;
 };
 // Plan for (m, n, k) on a device with sm_count SMs, using at most `budget` workspace bytes
 // (the bf16 copy of X itself is always needed).
-GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget);
-// tcgen05 bf16 GEMM: Y = bf16(X) . bf16(W_hat)^T, FP32 accumulation in tensor memory.
+GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budget,
+                      bool split = false);
+// tcgen05 GEMM with FP32 accumulation in tensor memory: Y = bf16(X) . bf16(W_hat)^T, or in
+// the split form Y = (X_hi + X_lo) . (W_hi + W_lo)^T with all four products.
 int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *workspace,
                    const GemmPlan &plan, cudaStream_t s, const DevInfo &dev);
 // Reads (and optionally clears) the device-side record of bounded waits that gave up on
