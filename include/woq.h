@@ -179,8 +179,10 @@ size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path);
  *        hold 64 activation rows, and one MMA per operand half multiplies the weight tile
  *        against both X halves, so all four products land in the FP32 accumulator. For
  *        int4, v_hi + v_lo == v exactly; x (and an int8 v) keeps 16 significand bits.
- *        Four times the tensor-core work of BF16_TC; meant for small batches (m <= 64)
- *        whose FP32 CUDA-core cost grows with m.
+ *        Four times the tensor-core work of BF16_TC; meant for small batches whose FP32
+ *        CUDA-core cost grows with m. One launch, no workspace (qgemm_workspace_bytes is 0):
+ *        the kernel converts X itself, and when K is split across CTAs those CTAs form one
+ *        thread-block cluster that sums the partials in shared memory, in a fixed order.
  *   path WOQ_PATH_FP32: the same FP32 arithmetic as qgemv, for any m.
  *   path WOQ_PATH_AUTO: BF16_TC if m >= 128, SPLIT_TC if 24 <= m < 128, else FP32.
  *   X  device, [m, k] float32 row-major, 16-byte aligned

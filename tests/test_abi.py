@@ -95,14 +95,14 @@ def test_workspace_sizing():
     assert L.qgemm_workspace_bytes(4, ctypes.byref(w), _lib.WOQ_PATH_FP32) == 0
     assert L.qgemm_workspace_bytes(4, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 0
     assert L.qgemm_workspace_bytes(23, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 0
-    assert L.qgemm_workspace_bytes(24, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 128 * 3072 * 2
+    assert L.qgemm_workspace_bytes(127, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 0
     assert L.qgemm_workspace_bytes(512, ctypes.byref(w), _lib.WOQ_PATH_AUTO) == 512 * 3072 * 2
     assert L.qgemm_workspace_bytes(375, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC) % 256 == 0
     assert L.qgemm_workspace_bytes(0, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC) == 0
     assert L.qgemm_workspace_bytes(16, ctypes.byref(_w(bits=3)), 0) == 0
-    # split form: 128 bf16 rows (hi then lo) per 64-row tile; no device -> no K-split partials
-    assert L.qgemm_workspace_bytes(4, ctypes.byref(w), _lib.WOQ_PATH_SPLIT_TC) == 128 * 3072 * 2
-    assert L.qgemm_workspace_bytes(65, ctypes.byref(w), _lib.WOQ_PATH_SPLIT_TC) == 256 * 3072 * 2
+    # split form: X tiles written in-kernel, K-split partials summed on chip -> no workspace
+    assert L.qgemm_workspace_bytes(4, ctypes.byref(w), _lib.WOQ_PATH_SPLIT_TC) == 0
+    assert L.qgemm_workspace_bytes(65, ctypes.byref(w), _lib.WOQ_PATH_SPLIT_TC) == 0
     assert L.qgemm_workspace_bytes(4, ctypes.byref(w), 4) == 0
 
 

@@ -107,11 +107,9 @@ def test_fp32_path_any_m(bits, m):
 def test_auto_path_picks_by_m():
     W = workloads.weight(256, 1024, seed=9)
     w, p, s = packed_from_weight(W, 4)
-    # below 24 rows: the CUDA-core kernel, no workspace
+    # below 128 rows: the CUDA-core kernel or the split tensor-core form, no workspace
     assert woq.qgemm_workspace_bytes(23, w, "auto") == 0
-    # 24..127 rows: the split tensor-core form, 128 bf16 rows (hi + lo) per 64-row tile
-    assert woq.qgemm_workspace_bytes(64, w, "auto") == woq.qgemm_workspace_bytes(64, w, "split_tc")
-    assert woq.qgemm_workspace_bytes(64, w, "auto") >= 128 * 1024 * 2
+    assert woq.qgemm_workspace_bytes(64, w, "auto") == 0
     # from 128 rows: the bf16 copy of X, plus FP32 partials when the plan splits K
     assert woq.qgemm_workspace_bytes(128, w, "auto") == woq.qgemm_workspace_bytes(128, w, "bf16_tc")
     for m in (8, 64):  # both FP32-accurate paths

@@ -88,30 +88,38 @@ def test_split_tc_lm_head_int8_sampled():
     assert max_rel(Y[:, rows], ref_rows(X.numpy(), p, s, 8, rows)) <= FP32_TOL
 
 
-def test_split_tc_workspace_and_determinism():
-    """Workspace covers 128 bf16 rows (hi + lo) per 64-row tile; repeated calls agree bitwise;
-    each call launches the X split, the GEMM and, when K is split, the reduction."""
-    n, k = 1024, 3072
-    W = workloads.weight(n, k, seed=12)
-    w, p, s = packed_from_weight(W, 4)
-    for m in (1, 64, 65):
-        assert woq.qgemm_workspace_bytes(m, w, "split_tc") >= ((m + 63) // 64) * 128 * k * 2
-    X = workloads.activations(64, k, seed=13).cuda()
-    ws = torch.empty(woq.qgemm_workspace_bytes(64, w, "split_tc"), dtype=torch.uint8, device="cuda")
-    before = woq.launch_count()
-    a = woq.qgemm(X, w, path="split_tc", workspace=ws)
-    b = woq.qgemm(X, w, path="split_tc", workspace=ws)
-    assert torch.equal(a, b)
-    assert woq.launch_count() - before in (4, 6)
-    assert woq.device_status() == 0
-    assert max_rel(a.cpu().numpy(), ref_rows(X.cpu().numpy(), p, s, 4)) <= FP32_TOL
+def test_split_tc_one_launch_no_workspace_deterministic():
+    """No workspace; one launch per call (K-splits summed inside their cluster); repeated calls
+    agree bitwise, with and without K-splits."""
+    for n, k in ((1024, 3072), (6144, 1024), (4096, 1024)):
+        W = workloads.weight(n, k, seed=12 + n)
+        w, p, s = packed_from_weight(W, 4)
+        for m in (1, 64, 65):
+            assert woq.qgemm_workspace_bytes(m, w, "split_tc") == 0
+        X = workloads.activations(64, k, seed=13).cuda()
+        before = woq.launch_count()
+        a = woq.qgemm(X, w, path="split_tc")
+        b = woq.qgemm(X, w, path="split_tc")
+        assert woq.launch_count() - before == 2
+        assert torch.equal(a, b)
+        assert woq.device_status() == 0
+        assert max_rel(a.cpu().numpy(), ref_rows(X.cpu().numpy(), p, s, 4)) <= FP32_TOL
 
 
-def test_split_tc_too_small_workspace_is_refused():
-    W = workloads.weight(256, 1024, seed=14)
-    w, _, _ = packed_from_weight(W, 4)
-    X = workloads.activations(16, 1024, seed=15).cuda()
-    need = woq.qgemm_workspace_bytes(16, w, "split_tc")
-    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
-    with pytest.raises(woq.WoqError):
-        woq.qgemm(X, w, path="split_tc", workspace=ws)
+def test_split_tc_in_a_cuda_graph():
+    """Captured and replayed: the cluster launch and its on-chip reduction replay correctly."""
+    n, k = 1024, 2048
+    W = workloads.weight(n, k, seed=16)
+    w, p, s = packed_from_weight(W, 8)
+    X = workloads.activations(48, k, seed=17).cuda()
+    Y = torch.empty(48, n, device="cuda")
+    woq.qgemm(X, w, path="split_tc", out=Y)  # warm-up outside the capture
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            woq.qgemm(X, w, path="split_tc", out=Y, stream=st)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert max_rel(Y.cpu().numpy(), ref_rows(X.cpu().numpy(), p, s, 8)) <= FP32_TOL

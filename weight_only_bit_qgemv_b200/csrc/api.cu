@@ -171,8 +171,10 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
   woq::GemmPlan plan;
   if (p != WOQ_PATH_FP32) {
     plan = woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX, p == WOQ_PATH_SPLIT_TC);
-    if (!workspace || workspace_bytes < plan.total) return WOQ_EWORKSPACE;
-    if (!woq::aligned(workspace, 256)) return WOQ_EALIGN;
+    if (plan.total > 0) {
+      if (!workspace || workspace_bytes < plan.total) return WOQ_EWORKSPACE;
+      if (!woq::aligned(workspace, 256)) return WOQ_EALIGN;
+    }
   }
   DevInfo dev;
   rc = woq::current_device(&dev);

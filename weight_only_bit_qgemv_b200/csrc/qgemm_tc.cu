@@ -69,7 +69,7 @@ long long g_wait_limit_cycles = 0;  // test hook: > 0 wait limit, < 0 inject a s
 
 struct Shared {
   uint64_t wfull[kMaxSL];   // raw code tile and X tile landed (TMA bytes)
-  uint64_t lempty[kMaxSL];  // load stage free: MMA commit + one arrival per dequant warp
+  uint64_t lempty[kMaxSL];  // load stage free: the stage's MMA commit (see the dequantisers)
   uint64_t bfull[kMaxSB];   // B tile written (one arrival per dequant warp)
   uint64_t bempty[kMaxSB];  // B tile read by the MMAs (commit)
   uint64_t sfull[2];        // scale tile landed (TMA bytes)
@@ -217,14 +217,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s, const uint16_t *__restrict__ scales,
                     float *__restrict__ Y, int M, int N, int K, int sl_stages, int sc_bytes,
-                    int sc_bufs, int splits, float *__restrict__ partials, long long wait_limit,
-                    long long stuck_wait) {
+                    int sc_bufs, int splits, float *__restrict__ partials,
+                    const float *__restrict__ Xf, long long wait_limit, long long stuck_wait) {
   constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
   constexpr int kRawBytes = BN * kRawRow;
   // SPLIT (FP32-accurate form): each X tile holds 64 activation rows as bf16 hi then bf16 lo
   // (128 rows), each weight slot holds the bf16 hi and lo tiles of the dequantised weights,
   // and per K-step two M=128, N=128 MMAs (A = weight hi, then weight lo; B = the X tile)
-  // accumulate all four products; the epilogue adds the hi and lo column halves.
+  // accumulate all four products; the epilogue adds the hi and lo column halves. The
+  // epilogue warps, idle during the main loop, also write the X tiles from FP32 X (no
+  // pre-pass), and the K-splits of one output tile run as one thread-block cluster that sums
+  // its partials through distributed shared memory (no workspace, no reduction launch).
+  // One work unit per CTA: the host launches one CTA per unit.
   static_assert(!SPLIT || (MH == 1 && BN == BM), "the split form uses 128-row weight tiles");
   constexpr bool kSwap = MH == 2 || SPLIT;       // A = weight tile, B = X tile
   constexpr int kBBytes1 = BN * BK * 2;          // one dequantised weight tile
@@ -262,8 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SL; ++s) {
-      ptx::mbar_init(&sh.wfull[s], 1);
-      ptx::mbar_init(&sh.lempty[s], 1 + kDequantWarps);  // MMA commit + dequant warps
+      // split form: the producer's byte count plus one arrival per epilogue warp (X written)
+      ptx::mbar_init(&sh.wfull[s], SPLIT ? 1 + kEpiWarps : 1);
+      ptx::mbar_init(&sh.lempty[s], 1);  // MMA commit
     }
     for (int s = 0; s < kSB; ++s) {
       ptx::mbar_init(&sh.bfull[s], kDequantWarps);
@@ -281,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&tm_x);
+    if (!SPLIT) ptx::prefetch_tmap(&tm_x);
     ptx::prefetch_tmap(&tm_w);
     if (sc_tma) ptx::prefetch_tmap(&tm_s);
   }
@@ -333,15 +338,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // Both copies of the stage complete on one barrier. The dequantisers wait on it and
           // only then mark their weight tile ready, so the MMA thread waits once per stage.
-          ptx::mbar_arrive_expect_tx(&sh.wfull[s], kRawBytes + kAStage);
+          ptx::mbar_arrive_expect_tx(&sh.wfull[s], SPLIT ? kRawBytes : kRawBytes + kAStage);
           ptx::tma_load_2d(smem + L.raw + s * kRawBytes, &tm_w, &sh.wfull[s], ks * kRawRow, nb * BN);
           wmask |= 1u << s;
           wpar = (wpar & ~(1u << s)) | (ph << s);
-          if (!waited) {
-            ptx::pdl_wait();
-            waited = true;
+          if constexpr (!SPLIT) {  // the split form's X tiles are written by the epilogue warps
+            if (!waited) {
+              ptx::pdl_wait();
+              waited = true;
+            }
+            ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.wfull[s], ks * BK, mb * kXRows);
           }
-          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.wfull[s], ks * BK, mb * kXRows);
           if (++s == SL) {
             s = 0;
             ph ^= 1;
@@ -502,13 +509,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // Each lane makes its writes visible to the async proxy (the tensor core), the warp
-        // converges, and one lane arrives for the warp.
+        // converges, and one lane arrives for the warp. The load stage needs no arrival from
+        // here: the MMA issuer waits for every warp's bfull arrival (each warp is done with
+        // the raw codes by then) before it issues, and frees the stage by its commit.
         ptx::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&sh.bfull[bs]);
-          ptx::mbar_arrive(&sh.lempty[s]);
-        }
+        if (lane == 0) ptx::mbar_arrive(&sh.bfull[bs]);
         if (++s == SL) {
           s = 0;
           ph ^= 1;
@@ -526,6 +532,97 @@ __global__ void __launch_bounds__(kThreads, 1)
           sph ^= 1;
         }
       }
+    }
+  } else if constexpr (SPLIT) {
+    // ---- split form, epilogue warps: write the X tiles, then accumulator -> Y ----
+    const int q = warp & 3;                                  // TMEM lanes 32q .. 32q+31
+    const int et = threadIdx.x - (2 + kDequantWarps) * 32;   // 0 .. 127
+    const int u = blockIdx.x;                                // one work unit per CTA
+    const int tile = u / splits, sp = u - tile * splits;
+    const int mb = tile % num_m, nb = tile / num_m;
+    const int ks0 = sp * kps, ks1 = min(num_k, ks0 + kps);
+    const int rows = min(TM, M - mb * TM);                   // activation rows of the tile
+    const int n0 = nb * BN;
+    bool ok = u < num_units;
+    ptx::pdl_wait();  // X is written, and Y may be read, by preceding kernels
+    // (1) X tiles: 64 FP32 rows -> bf16 hi in tile rows 0..63 and bf16 lo in rows 64..127,
+    // in the 128-byte-swizzled order a TMA copy would produce. Columns past K are zero
+    // (K % 32 == 0, so an 8-column chunk is wholly inside or outside). Tile rows past the
+    // last activation row are left as they are: they only feed accumulator columns that are
+    // never read.
+    {
+      const float *xt = Xf + static_cast<size_t>(mb * TM) * K;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ks = ks0; ks < ks1 && ok; ++ks) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.lempty[s], ph ^ 1, wait_limit, abort))) {
+          record_timeout(abort);
+          ok = false;
+          break;
+        }
+        uint8_t *xs = smem + L.a + s * kAStage;
+        for (int job = et; job < rows * 8; job += kEpiWarps * 32) {
+          const int r = job >> 3, c = job & 7;
+          const int col = ks * BK + c * 8;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+          if (col < K) {
+            const float4 *src = reinterpret_cast<const float4 *>(xt + static_cast<size_t>(r) * K + col);
+            a = __ldg(src);
+            b = __ldg(src + 1);
+          }
+          uint4 h, l;
+          split_pack(a.x, a.y, h.x, l.x);
+          split_pack(a.z, a.w, h.y, l.y);
+          split_pack(b.x, b.y, h.z, l.z);
+          split_pack(b.z, b.w, h.w, l.w);
+          const int off = (c ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4 *>(xs + r * 128 + off) = h;
+          *reinterpret_cast<uint4 *>(xs + (TM + r) * 128 + off) = l;
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.wfull[s]);
+        if (++s == SL) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+    }
+    // (2) Accumulator: TMEM lane = weight row, column t = activation row t's hi part, column
+    // 64 + t its lo part; their sum goes to Y (one split) or to this CTA's staged partial
+    // [64][BN] in the X ring, now idle (every MMA, the only reader, has completed), which
+    // the cluster sums after the roles end.
+    if (ok && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.accfull[0], 0, wait_limit, abort,
+                                                              kRoleSleepNs))) {
+      record_timeout(abort);
+      ok = false;
+    }
+    float *stage = reinterpret_cast<float *>(smem + L.a);
+    if (ok) {
+      ptx::tc_fence_after();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const int nl = q * 32 + lane;
+      for (int c0 = 0; c0 < rows; c0 += 16) {  // warp-uniform trip count
+        uint32_t ra[16], rb[16];
+        ptx::tmem_ld_32x32b_x16(tb + c0, ra);
+        ptx::tmem_ld_32x32b_x16(tb + TM + c0, rb);
+        ptx::tmem_ld_wait(ra);
+        ptx::tmem_ld_wait(rb);
+        if (splits == 1) {
+          // for each activation row the warp's lanes store 32 consecutive floats of Y
+          float *p = Y + static_cast<size_t>(mb * TM + c0) * N + n0 + nl;
+          if (n0 + nl < N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j, p += N)
+              if (c0 + j < rows) *p = __uint_as_float(ra[j]) + __uint_as_float(rb[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < rows) stage[(c0 + j) * BN + nl] = __uint_as_float(ra[j]) + __uint_as_float(rb[j]);
+        }
+      }
+      ptx::tc_fence_before();
     }
   } else {
     // ---- epilogue: TMEM accumulator -> registers -> Y ----
@@ -550,79 +647,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int n0 = nb * BN;
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * kAccCols;
-      if constexpr (SPLIT) {
-        // TMEM lane = weight row n; column t holds the token's hi part, column 64 + t its lo
-        // part: Y[m][n] is their sum. Each 16-column chunk loads both halves.
-        const int n = n0 + q * 32 + lane;
-        const int ncols = min(TM, M - mb * TM);
-        for (int c0 = 0; c0 < ncols; c0 += 16) {  // warp-uniform trip count
-          uint32_t ra[16], rb[16];
-          ptx::tmem_ld_32x32b_x16(tb + c0, ra);
-          ptx::tmem_ld_32x32b_x16(tb + TM + c0, rb);
-          ptx::tmem_ld_wait(ra);
-          ptx::tmem_ld_wait(rb);
-          const int mrem = ncols - c0;
+      // 16-column chunks, software-pipelined: the next chunk's TMEM load is in flight while
+      // this one is stored (two register buffers, each waited for before use).
+      const int ncols = MH == 2 ? min(TM, M - mb * TM) : BN;
+      const int nchunks = (ncols + 15) / 16;
+      auto store_chunk = [&](const uint32_t (&r)[16], int c) {
+        const int c0 = 16 * c;
+        if constexpr (MH == 2) {
+          // TMEM lane = weight row n, column = activation row m: for each column the warp's
+          // 32 lanes store 32 consecutive floats of one Y row. The row pointer advances by
+          // N per column; full chunks skip the row check.
+          const int n = n0 + q * 32 + lane;
+          const int mrem = M - (mb * TM + c0);
           float *p = out + static_cast<size_t>(mb * TM + c0) * N + n;
           if (n < N) {
+            if (mrem >= 16) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j, p += N)
-              if (j < mrem) *p = __uint_as_float(ra[j]) + __uint_as_float(rb[j]);
+              for (int j = 0; j < 16; ++j, p += N) *p = __uint_as_float(r[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j, p += N)
+                if (j < mrem) *p = __uint_as_float(r[j]);
+            }
+          }
+        } else {
+          const int grow = mb * TM + q * 32 + lane;
+          if (grow < M) {
+            float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
+            if (vec && n0 + c0 + 16 <= N) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                reinterpret_cast<float4 *>(yr)[v] =
+                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            } else {
+#pragma unroll
+              for (int v = 0; v < 16; ++v)
+                if (n0 + c0 + v < N) yr[v] = __uint_as_float(r[v]);
+            }
           }
         }
-      } else {
-        // 16-column chunks, software-pipelined: the next chunk's TMEM load is in flight while
-        // this one is stored (two register buffers, each waited for before use).
-        const int ncols = MH == 2 ? min(TM, M - mb * TM) : BN;
-        const int nchunks = (ncols + 15) / 16;
-        auto store_chunk = [&](const uint32_t (&r)[16], int c) {
-          const int c0 = 16 * c;
-          if constexpr (MH == 2) {
-            // TMEM lane = weight row n, column = activation row m: for each column the warp's
-            // 32 lanes store 32 consecutive floats of one Y row. The row pointer advances by
-            // N per column; full chunks skip the row check.
-            const int n = n0 + q * 32 + lane;
-            const int mrem = M - (mb * TM + c0);
-            float *p = out + static_cast<size_t>(mb * TM + c0) * N + n;
-            if (n < N) {
-              if (mrem >= 16) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j, p += N) *p = __uint_as_float(r[j]);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j, p += N)
-                  if (j < mrem) *p = __uint_as_float(r[j]);
-              }
-            }
-          } else {
-            const int grow = mb * TM + q * 32 + lane;
-            if (grow < M) {
-              float *yr = out + static_cast<size_t>(grow) * N + n0 + c0;
-              if (vec && n0 + c0 + 16 <= N) {
-#pragma unroll
-                for (int v = 0; v < 4; ++v)
-                  reinterpret_cast<float4 *>(yr)[v] =
-                      make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                  __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-              } else {
-#pragma unroll
-                for (int v = 0; v < 16; ++v)
-                  if (n0 + c0 + v < N) yr[v] = __uint_as_float(r[v]);
-              }
-            }
-          }
-        };
-        uint32_t ra[16], rb[16];
-        ptx::tmem_ld_32x32b_x16(tb, ra);
-        ptx::tmem_ld_wait(ra);
-        for (int c = 0; c < nchunks; c += 2) {  // trip counts are warp-uniform
-          if (c + 1 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 1), rb);
-          store_chunk(ra, c);
-          if (c + 1 < nchunks) {
-            ptx::tmem_ld_wait(rb);
-            if (c + 2 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 2), ra);
-            store_chunk(rb, c + 1);
-            if (c + 2 < nchunks) ptx::tmem_ld_wait(ra);
-          }
+      };
+      uint32_t ra[16], rb[16];
+      ptx::tmem_ld_32x32b_x16(tb, ra);
+      ptx::tmem_ld_wait(ra);
+      for (int c = 0; c < nchunks; c += 2) {  // trip counts are warp-uniform
+        if (c + 1 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 1), rb);
+        store_chunk(ra, c);
+        if (c + 1 < nchunks) {
+          ptx::tmem_ld_wait(rb);
+          if (c + 2 < nchunks) ptx::tmem_ld_32x32b_x16(tb + 16 * (c + 2), ra);
+          store_chunk(rb, c + 1);
+          if (c + 2 < nchunks) ptx::tmem_ld_wait(ra);
         }
       }
       ptx::tc_fence_before();
@@ -632,6 +708,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         ab = 0;
         aph ^= 1;
       }
+    }
+  }
+
+  if constexpr (SPLIT) {
+    // Several K-splits: the cluster's CTAs (rank = split) sum their staged partials through
+    // distributed shared memory, every thread of the cluster taking part. The cluster
+    // barriers make the staged partials visible before the reads and keep every CTA (and
+    // its shared memory) alive until all reads are done. Every thread arrives whatever its
+    // role did before, and every role's waits are bounded, so the barriers are reached.
+    if (splits > 1) {
+      ptx::cluster_sync();
+      ptx::pdl_wait();  // Y may be read by preceding kernels (passed already by the epilogue)
+      const int u = blockIdx.x;
+      const int tile = u / splits, sp = u - tile * splits;
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int rows = min(TM, M - mb * TM);
+      const int per = (rows + splits - 1) / splits;  // activation rows summed by this CTA
+      const int j0 = sp * per, j1 = min(rows, j0 + per);
+      const uint32_t st = ptx::smem_u32(smem + L.a);
+      const bool vec = (N & 3) == 0;
+      for (int i = threadIdx.x; i < (j1 - j0) * (BN / 4); i += kThreads) {
+        const int j = j0 + i / (BN / 4), c4 = i % (BN / 4);
+        const uint32_t off = static_cast<uint32_t>((j * BN + 4 * c4) * 4);
+        float4 acc = ptx::ld_shared_cluster_v4(ptx::mapa_shared(st + off, 0));
+        for (int r = 1; r < splits; ++r) {
+          const float4 v = ptx::ld_shared_cluster_v4(ptx::mapa_shared(st + off, r));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int n = nb * BN + 4 * c4;
+        float *yr = Y + static_cast<size_t>(mb * TM + j) * N + n;
+        if (vec && n + 4 <= N) {
+          *reinterpret_cast<float4 *>(yr) = acc;
+        } else {
+          if (n < N) yr[0] = acc.x;
+          if (n + 1 < N) yr[1] = acc.y;
+          if (n + 2 < N) yr[2] = acc.z;
+          if (n + 3 < N) yr[3] = acc.w;
+        }
+      }
+      ptx::cluster_sync();
     }
   }
 
@@ -675,27 +794,6 @@ __global__ void __launch_bounds__(256) x_to_bf16_kernel(const float4 *__restrict
     t = __floats2bfloat162_rn(b.x, b.y); o.z = *reinterpret_cast<uint32_t *>(&t);
     t = __floats2bfloat162_rn(b.z, b.w); o.w = *reinterpret_cast<uint32_t *>(&t);
     xb[i] = o;
-  }
-}
-
-// X fp32 [m, k] -> per 64-token tile t, workspace rows 128t .. 128t+63 = bf16 hi = RNE(x)
-// and rows 128t+64 .. 128t+127 = bf16 lo = RNE(x - hi); 8 elements per thread.
-__global__ void __launch_bounds__(256) x_split_kernel(const float4 *__restrict__ x,
-                                                      uint4 *__restrict__ xs, int k8, size_t n8) {
-  ptx::pdl_wait();
-  ptx::pdl_launch_dependents();
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t row = i / k8, col = i - row * k8;
-    const float4 a = x[2 * i], b = x[2 * i + 1];
-    uint4 h, l;
-    split_pack(a.x, a.y, h.x, l.x);
-    split_pack(a.z, a.w, h.y, l.y);
-    split_pack(b.x, b.y, h.z, l.z);
-    split_pack(b.z, b.w, h.w, l.w);
-    const size_t base = (row / 64) * 128 + (row % 64);
-    xs[base * k8 + col] = h;
-    xs[(base + 64) * k8 + col] = l;
   }
 }
 
@@ -775,13 +873,14 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   if (sl < 2) return WOQ_ESHAPE;
   const int smem = make_layout(BITS, BN, kAStage, kBSlot, kSB, sl, sc_bytes, sc_bufs).total;
 
-  // The split form's workspace holds 128 rows (hi, then lo) per 64-token tile.
   const int64_t num_m = (m + TM - 1) / TM;
-  const int64_t x_rows = SPLIT ? num_m * kXRows : m;
   CUtensorMap tm_x, tm_w, tm_s;
-  if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, x_rows, BK,
-                          kXRows, CU_TENSOR_MAP_SWIZZLE_128B))
+  if constexpr (SPLIT) {  // the kernel writes its X tiles itself
+    std::memset(&tm_x, 0, sizeof(tm_x));
+  } else if (!make_tensor_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, w.k, m, BK,
+                                 kXRows, CU_TENSOR_MAP_SWIZZLE_128B)) {
     return WOQ_ECUDA;
+  }
   if (!make_tensor_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, w.k * BITS / 8, w.n,
                 BK * BITS / 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return WOQ_ECUDA;
@@ -793,11 +892,39 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
     std::memset(&tm_s, 0, sizeof(tm_s));
   }
 
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const long long lim = g_wait_limit_cycles > 0 ? g_wait_limit_cycles : kDefaultWaitLimit;
+  const long long stuck = g_wait_limit_cycles < 0 ? -g_wait_limit_cycles : 0;
+  const int64_t units = num_m * ((w.n + BN - 1) / BN) * plan.splits;
 
-  // 1) X -> bf16 (or bf16 hi + lo) into the workspace.
+  if constexpr (SPLIT) {
+    // One CTA per work unit; the K-splits of an output tile form one cluster.
+    if (units > INT32_MAX) return WOQ_ESHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (plan.splits > 1) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = static_cast<unsigned>(plan.splits);
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.numAttrs = 2;
+    }
+    if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_s, w.scales, Y, static_cast<int>(m),
+                           static_cast<int>(w.n), static_cast<int>(w.k), sl, sc_bytes, sc_bufs,
+                           plan.splits, static_cast<float *>(nullptr), X, lim, stuck) != cudaSuccess)
+      return WOQ_ECUDA;
+    count_launches(1);
+    return WOQ_OK;
+  }
+
+  // 1) X -> bf16 into the workspace.
   const size_t n8 = static_cast<size_t>(m) * w.k / 8;
   {
     cudaLaunchConfig_t cfg = {};
@@ -808,32 +935,25 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e;
-    if constexpr (SPLIT)
-      e = cudaLaunchKernelEx(&cfg, x_split_kernel, reinterpret_cast<const float4 *>(X),
-                             reinterpret_cast<uint4 *>(workspace), static_cast<int>(w.k / 8), n8);
-    else
-      e = cudaLaunchKernelEx(&cfg, x_to_bf16_kernel, reinterpret_cast<const float4 *>(X),
-                             reinterpret_cast<uint4 *>(workspace), n8);
-    if (e != cudaSuccess) return WOQ_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, x_to_bf16_kernel, reinterpret_cast<const float4 *>(X),
+                           reinterpret_cast<uint4 *>(workspace), n8) != cudaSuccess)
+      return WOQ_ECUDA;
     count_launches(1);
   }
   // 2) the persistent GEMM: one CTA per SM (or per work unit, if fewer).
   float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + plan.xb);
   {
-    const int64_t tiles = num_m * ((w.n + BN - 1) / BN) * plan.splits;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(tiles, dev.sm_count)), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(units, dev.sm_count)), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const long long lim = g_wait_limit_cycles > 0 ? g_wait_limit_cycles : kDefaultWaitLimit;
-    const long long stuck = g_wait_limit_cycles < 0 ? -g_wait_limit_cycles : 0;
     if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_s, w.scales, Y, static_cast<int>(m),
                            static_cast<int>(w.n), static_cast<int>(w.k), sl, sc_bytes, sc_bufs,
-                           plan.splits, partials, lim, stuck) != cudaSuccess)
+                           plan.splits, partials, static_cast<const float *>(nullptr), lim,
+                           stuck) != cudaSuccess)
       return WOQ_ECUDA;
     count_launches(1);
   }
@@ -880,30 +1000,33 @@ GemmPlan plan_gemm_tc(int64_t m, int64_t n, int64_t k, int sm_count, size_t budg
   GemmPlan p;
   p.split = split;
   const int64_t num_k = (k + BK - 1) / BK;
-  int64_t mt;
-  if (split) {
-    // 64-token tiles; the workspace holds 128 rows (hi, then lo) per tile.
-    mt = (m + 63) / 64;
-    p.xb = align(static_cast<size_t>(mt) * 128 * static_cast<size_t>(k) * 2);
-  } else {
-    // Past one 128-row M tile, 256 x 128 tiles (two M halves sharing each dequantised
-    // weight tile) halve the dequantisation per FLOP. Otherwise 128 x 256 tiles, which do
-    // twice the work per MMA instruction, when N allows.
-    p.xb = align(static_cast<size_t>(m) * static_cast<size_t>(k) * 2);
-    p.mh = m > 128 ? 2 : 1;
-    p.bn = p.mh == 1 && n >= 256 ? 256 : 128;
-    mt = (m + 128 * p.mh - 1) / (128 * p.mh);
-  }
-  int64_t tiles = mt * ((n + p.bn - 1) / p.bn);
-  // Split K until the work units cover the SMs, keeping >= 4 K-stages per split; the splits
-  // need FP32 partials in the workspace and a vectorisable Y (n % 4 == 0).
-  p.splits = 1;
-  if (n % 4 == 0 && sm_count > 0) {
-    while (p.splits < 8 && tiles * p.splits * 2 <= sm_count + sm_count / 4 &&
-           num_k / (p.splits * 2) >= 4 &&
-           p.xb + align(static_cast<size_t>(p.splits) * 2 * m * n * 4) <= budget)
+  // Work units cover the SMs: split K (at most 8 ways) while the units stay within 1.25x the
+  // SM count and every split keeps >= 4 K-stages.
+  auto grow_splits = [&](int64_t tiles, auto &&fits) {
+    while (p.splits < 8 && sm_count > 0 && tiles * p.splits * 2 <= sm_count + sm_count / 4 &&
+           num_k / (p.splits * 2) >= 4 && fits(p.splits * 2))
       p.splits *= 2;
+  };
+  if (split) {
+    // 64-row tiles; the kernel writes its own X tiles and a tile's K-splits (a cluster of at
+    // most 8, the portable size) sum their partials on chip: no workspace.
+    const int64_t tiles = ((m + 63) / 64) * ((n + 127) / 128);
+    grow_splits(tiles, [](int) { return true; });
+    return p;
   }
+  p.xb = align(static_cast<size_t>(m) * static_cast<size_t>(k) * 2);
+  // Past one 128-row M tile, 256 x 128 tiles (two M halves sharing each dequantised weight
+  // tile) halve the dequantisation per FLOP. Otherwise 128 x 256 tiles, which do twice the
+  // work per MMA instruction, when N allows.
+  p.mh = m > 128 ? 2 : 1;
+  p.bn = p.mh == 1 && n >= 256 ? 256 : 128;
+  const int64_t mt = (m + 128 * p.mh - 1) / (128 * p.mh);
+  const int64_t tiles = mt * ((n + p.bn - 1) / p.bn);
+  // The splits need FP32 partials in the workspace and a vectorisable Y (n % 4 == 0).
+  if (n % 4 == 0)
+    grow_splits(tiles, [&](int sp) {
+      return p.xb + align(static_cast<size_t>(sp) * m * n * 4) <= budget;
+    });
   if (p.splits == 1 && p.bn == 256 && tiles * 2 <= sm_count) p.bn = 128;  // more tiles instead
   p.part = p.splits > 1 ? align(static_cast<size_t>(p.splits) * m * n * 4) : 0;
   p.total = p.xb + p.part;
