@@ -5,19 +5,24 @@
 // read by the tensor core for all 128 rows of the M-tile.
 //
 // Persistent, warp-specialised kernel; one CTA per SM walks (128 * MH) x BN output tiles.
-//   warp 0        producer: bulk tensor copies (TMA, no multicast) of the bf16 X tile
-//                 (128B-swizzled, 128 * MH rows) and the raw code tile into a ring of SL load
-//                 stages, and of each output tile's [BN, K/32] scale tile into a double buffer
+//   warp 0        weight producer: bulk tensor copies (TMA, no multicast) of the raw code
+//                 tiles into a deep ring (up to 8 stages, freed by the dequantisers), and of
+//                 each output tile's [BN, K/32] scale tile into a double buffer
 //   warp 1        TMEM owner; one thread issues tcgen05.mma (K=16, bf16 x bf16 -> f32) into
 //                 one of two accumulator sets and commits completions: M=128 activation rows x
 //                 N=BN for MH = 1; for MH = 2 the operands swap, M=128 weight rows x N=256
 //                 activation rows
-//   warps 2..17   dequantisers: raw codes + binary16 scales -> bf16(scale * code) written
+//   warp 2        X producer: TMA copies of the bf16 X tile (128B-swizzled, 128 * MH rows)
+//                 into a ring of up to 4 stages, freed by the MMA commits
+//   warps 3..18   dequantisers: raw codes + binary16 scales -> bf16(scale * code) written
 //                 into a short ring of B tiles in the 128B-swizzled K-major layout that the
 //                 MMA's shared-memory descriptor names; with MH = 2 each weight tile meets 256
 //                 activation rows, so the dequantisation per FLOP is halved
-//   warps 18..21  epilogue: tcgen05.ld of the finished accumulators -> FP32 Y, while the MMA
+//   warps 19..22  epilogue: tcgen05.ld of the finished accumulators -> FP32 Y, while the MMA
 //                 thread already fills the other set with the next tile
+// Raw codes and X tiles travel in separate rings so that each is freed by its own reader:
+// a shared load slot could only be reused once the MMAs had read its X tile, which held
+// the raw codes (and with them the dequantisers) to the MMAs' pace.
 // Every mbarrier wait is bounded. A wait that gives up records the event in a device flag
 // and stops the CTA's other roles; the CTA drains the copies and MMAs it issued, frees
 // tensor memory and returns.
@@ -39,18 +44,26 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;              // bf16 elements per stage = one 128-byte swizzle row
-constexpr int kMaxSL = 8;           // load stages (X tile + raw code tile)
-constexpr int kMaxSB = 4;           // dequantised weight tiles (ring), at most
-// Weight-tile ring depth: 4 for 128-row tiles (the dequantisers then run two stages ahead
-// of the MMAs instead of waiting on each stage's completion), 2 for 256-row tiles.
+// Three rings, each freed by its own consumer: raw code tiles (read by the dequantisers),
+// X tiles (read by the MMAs) and dequantised weight tiles (written by the dequantisers, read
+// by the MMAs). Raw codes are small, so their ring is deep and the dequantisers never wait
+// for the MMAs to free a load slot.
+constexpr int kMaxSW = 8;  // raw code stages
+constexpr int kMaxSX = 4;  // X stages
+constexpr int kMaxSB = 3;  // dequantised weight tiles
+// Weight-tile ring depth: the dequantisers run up to this many K-steps ahead of the MMAs.
 __host__ __device__ constexpr int sb_for(int bn, bool split = false) {
-  return split ? 3 : bn == 128 ? 4 : 2;
+  return split || bn == 128 ? 3 : 2;
 }
 constexpr int kTmaScaleCols = 128;  // scale tile copied by TMA when K/32 <= this (and % 8 == 0)
 constexpr int kDequantWarps = 16;  // four per scheduler: each warp's chain is latency-bound
 constexpr int kDequantThreads = kDequantWarps * 32;
 constexpr int kEpiWarps = 4;
-constexpr int kThreads = (2 + kDequantWarps + kEpiWarps) * 32;  // 704
+// warp 0: raw-code and scale producer; 1: MMA issuer; 2: X producer; then the dequantisers,
+// then the epilogue warps
+constexpr int kDequantWarp0 = 3;
+constexpr int kEpiWarp0 = kDequantWarp0 + kDequantWarps;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;  // 736
 constexpr long long kDrainLimit = 1LL << 31;                    // cycles (~1 s)
 constexpr long long kDefaultWaitLimit = 1LL << 32;              // cycles (~2 s)
 constexpr int kSmemMax = 227 * 1024;
@@ -68,8 +81,10 @@ __host__ __device__ constexpr uint32_t idesc_for(int n) {
 long long g_wait_limit_cycles = 0;  // test hook: > 0 wait limit, < 0 inject a stuck wait
 
 struct Shared {
-  uint64_t wfull[kMaxSL];   // raw code tile and X tile landed (TMA bytes)
-  uint64_t lempty[kMaxSL];  // load stage free: the stage's MMA commit (see the dequantisers)
+  uint64_t wfull[kMaxSW];   // raw code tile landed (TMA bytes)
+  uint64_t wempty[kMaxSW];  // raw code tile read (one arrival per dequant warp)
+  uint64_t xfull[kMaxSX];   // X tile landed (TMA bytes; split form: one arrival per epilogue warp)
+  uint64_t xempty[kMaxSX];  // X tile read by the MMAs (commit)
   uint64_t bfull[kMaxSB];   // B tile written (one arrival per dequant warp)
   uint64_t bempty[kMaxSB];  // B tile read by the MMAs (commit)
   uint64_t sfull[2];        // scale tile landed (TMA bytes)
@@ -82,18 +97,18 @@ struct Shared {
   int abort;
 };
 
-// Shared-memory layout for a given number of load stages and scale-tile size.
+// Shared-memory layout for given ring depths and scale-tile size.
 struct Layout {
   int a, b, raw, sc, bar, total;
 };
 __host__ __device__ inline Layout make_layout(int bits, int bn, int x_stage, int b_slot, int sb,
-                                              int sl, int sc_bytes, int sc_bufs) {
+                                              int sx, int sw, int sc_bytes, int sc_bufs) {
   Layout L;
   const int raw_bytes = bn * BK * bits / 8;
   L.a = 0;
-  L.b = L.a + sl * x_stage;
+  L.b = L.a + sx * x_stage;
   L.raw = L.b + sb * b_slot;
-  L.sc = L.raw + sl * raw_bytes;
+  L.sc = L.raw + sw * raw_bytes;
   L.bar = (L.sc + sc_bufs * sc_bytes + 127) & ~127;
   L.total = L.bar + static_cast<int>(sizeof(Shared)) + 1024;  // + base alignment slack
   return L;
@@ -216,8 +231,8 @@ template <int BITS, int BN, int MH, bool SPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_s, const uint16_t *__restrict__ scales,
-                    float *__restrict__ Y, int M, int N, int K, int sl_stages, int sc_bytes,
-                    int sc_bufs, int splits, float *__restrict__ partials,
+                    float *__restrict__ Y, int M, int N, int K, int sx_stages, int sw_stages,
+                    int sc_bytes, int sc_bufs, int splits, float *__restrict__ partials,
                     const float *__restrict__ Xf, long long wait_limit, long long stuck_wait) {
   constexpr int kRawRow = BK * BITS / 8;  // bytes of one row's codes per stage
   constexpr int kRawBytes = BN * kRawRow;
@@ -247,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kTmemCols = 2 * kAccCols;   // two accumulator sets
   static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
   constexpr uint32_t kIdesc = idesc_for(kAccCols);
-  const Layout L = make_layout(BITS, BN, kAStage, kBBytes, kSB, sl_stages, sc_bytes, sc_bufs);
+  const Layout L = make_layout(BITS, BN, kAStage, kBBytes, kSB, sx_stages, sw_stages, sc_bytes, sc_bufs);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -262,13 +277,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Work unit u covers output tile u / splits and K-stages [ks0, ks1) of split u % splits.
   const int num_units = num_m * ((N + BN - 1) / BN) * splits;
   const int kps = (num_k + splits - 1) / splits;
-  const int SL = sl_stages;
+  const int SX = sx_stages, SW = sw_stages;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SL; ++s) {
-      // split form: the producer's byte count plus one arrival per epilogue warp (X written)
-      ptx::mbar_init(&sh.wfull[s], SPLIT ? 1 + kEpiWarps : 1);
-      ptx::mbar_init(&sh.lempty[s], 1);  // MMA commit
+    for (int s = 0; s < SW; ++s) {
+      ptx::mbar_init(&sh.wfull[s], 1);
+      ptx::mbar_init(&sh.wempty[s], kDequantWarps);
+    }
+    for (int s = 0; s < SX; ++s) {
+      ptx::mbar_init(&sh.xfull[s], SPLIT ? kEpiWarps : 1);
+      ptx::mbar_init(&sh.xempty[s], 1);
     }
     for (int s = 0; s < kSB; ++s) {
       ptx::mbar_init(&sh.bfull[s], kDequantWarps);
@@ -301,20 +319,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // producer bookkeeping for the drain: slots issued at least once, and the parity of
   // their last issue
-  uint32_t wmask = 0, wpar = 0, smask = 0, spar = 0;
+  uint32_t wmask = 0, wpar = 0, smask = 0, spar = 0, xmask = 0, xpar = 0;
   bool mma_issued = false;
 
   if (warp == 0) {
-    // ---- producer (one lane). Only X depends on preceding kernels: wait before it. ----
+    // ---- raw-code and scale producer (one lane): weights only, no wait on preceding grids.
     // Ring positions advance incrementally (no division on the issue path); a wait with the
     // opposite parity passes at once on a fresh barrier, so the first round needs no case.
     if (lane == 0) {
       int s = 0, sb = 0;
       uint32_t ph = 0, sph = 0;
-      bool waited = false, ok = true;
+      bool ok = true;
       for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
         const int tile = u / splits, sp = u - (u / splits) * splits;
-        const int mb = tile % num_m, nb = tile / num_m;
+        const int nb = tile / num_m;
         const int ks0 = sp * kps, ks1 = min(num_k, ks0 + kps);
         if (sc_tma) {
           if (!ptx::mbar_wait_bounded(&sh.sempty[sb], sph ^ 1, wait_limit, abort, kRoleSleepNs)) {
@@ -331,25 +349,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         for (int ks = ks0; ks < ks1; ++ks) {
-          if (!ptx::mbar_wait_bounded(&sh.lempty[s], ph ^ 1, wait_limit, abort, kRoleSleepNs)) {
+          if (!ptx::mbar_wait_bounded(&sh.wempty[s], ph ^ 1, wait_limit, abort, kRoleSleepNs)) {
             record_timeout(abort);
             ok = false;
             break;
           }
-          // Both copies of the stage complete on one barrier. The dequantisers wait on it and
-          // only then mark their weight tile ready, so the MMA thread waits once per stage.
-          ptx::mbar_arrive_expect_tx(&sh.wfull[s], SPLIT ? kRawBytes : kRawBytes + kAStage);
+          ptx::mbar_arrive_expect_tx(&sh.wfull[s], kRawBytes);
           ptx::tma_load_2d(smem + L.raw + s * kRawBytes, &tm_w, &sh.wfull[s], ks * kRawRow, nb * BN);
           wmask |= 1u << s;
           wpar = (wpar & ~(1u << s)) | (ph << s);
-          if constexpr (!SPLIT) {  // the split form's X tiles are written by the epilogue warps
-            if (!waited) {
-              ptx::pdl_wait();
-              waited = true;
-            }
-            ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.wfull[s], ks * BK, mb * kXRows);
+          if (++s == SW) {
+            s = 0;
+            ph ^= 1;
           }
-          if (++s == SL) {
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ---- X producer (one lane; the split form's X tiles are written by the epilogue warps).
+    // X is written by preceding kernels: wait for them before the first copy.
+    if (!SPLIT && lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      ptx::pdl_wait();
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const int tile = u / splits, sp = u - (u / splits) * splits;
+        const int mb = tile % num_m;
+        const int ks0 = sp * kps, ks1 = min(num_k, ks0 + kps);
+        for (int ks = ks0; ks < ks1; ++ks) {
+          if (!ptx::mbar_wait_bounded(&sh.xempty[s], ph ^ 1, wait_limit, abort)) {
+            record_timeout(abort);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&sh.xfull[s], kAStage);
+          ptx::tma_load_2d(smem + L.a + s * kAStage, &tm_x, &sh.xfull[s], ks * BK, mb * kXRows);
+          xmask |= 1u << s;
+          xpar = (xpar & ~(1u << s)) | (ph << s);
+          if (++s == SX) {
             s = 0;
             ph ^= 1;
           }
@@ -378,9 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(ab * kAccCols);
         for (int ks = ks0; ks < ks1; ++ks) {
-          // bfull completes after every dequantiser has seen this stage's copies land (X and
-          // the raw codes share wfull), so it covers the X tile as well.
-          ok = ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort);
+          ok = ptx::mbar_wait_bounded(&sh.bfull[bs], bph, wait_limit, abort) &&
+               ptx::mbar_wait_bounded(&sh.xfull[s], ph, wait_limit, abort);
           if (!ok) {
             record_timeout(abort);
             break;
@@ -403,9 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           mma_issued = true;
-          ptx::tc_commit(&sh.lempty[s]);
+          ptx::tc_commit(&sh.xempty[s]);
           ptx::tc_commit(&sh.bempty[bs]);
-          if (++s == SL) {
+          if (++s == SX) {
             s = 0;
             ph ^= 1;
           }
@@ -423,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_commit(&sh.drain);  // arrives once every MMA issued above has completed
     }
-  } else if (warp < 2 + kDequantWarps) {
+  } else if (warp < kEpiWarp0) {
     // ---- dequantisers: 512 threads, one job of E codes per stage each: part t % P of row
     //      t / P, P = 64 / E parts per row (E = 32 at BN = 256, 16 at BN = 128). A warp's lanes
     //      cover 32 / P whole rows, so their raw-code loads are one contiguous range and their
@@ -431,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int E = BN * BK / kDequantThreads;  // codes per job
     constexpr int CH = E / 8;                     // 16-byte B chunks per job
     constexpr int P = BK / E;                     // jobs per row
-    const int t = threadIdx.x - 64;
+    const int t = threadIdx.x - kDequantWarp0 * 32;
     const int row = t / P, part = t % P;
     const int spr = K >> 5;
     const int sw = row & 7;
@@ -509,13 +546,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // Each lane makes its writes visible to the async proxy (the tensor core), the warp
-        // converges, and one lane arrives for the warp. The load stage needs no arrival from
-        // here: the MMA issuer waits for every warp's bfull arrival (each warp is done with
-        // the raw codes by then) before it issues, and frees the stage by its commit.
+        // converges, and one lane arrives for the warp: its B rows are written and its raw
+        // codes read.
         ptx::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.bfull[bs]);
-        if (++s == SL) {
+        if (lane == 0) {
+          ptx::mbar_arrive(&sh.bfull[bs]);
+          ptx::mbar_arrive(&sh.wempty[s]);
+        }
+        if (++s == SW) {
           s = 0;
           ph ^= 1;
         }
@@ -536,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if constexpr (SPLIT) {
     // ---- split form, epilogue warps: write the X tiles, then accumulator -> Y ----
     const int q = warp & 3;                                  // TMEM lanes 32q .. 32q+31
-    const int et = threadIdx.x - (2 + kDequantWarps) * 32;   // 0 .. 127
+    const int et = threadIdx.x - kEpiWarp0 * 32;             // 0 .. 127
     const int u = blockIdx.x;                                // one work unit per CTA
     const int tile = u / splits, sp = u - tile * splits;
     const int mb = tile % num_m, nb = tile / num_m;
@@ -555,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       for (int ks = ks0; ks < ks1 && ok; ++ks) {
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.lempty[s], ph ^ 1, wait_limit, abort))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.xempty[s], ph ^ 1, wait_limit, abort))) {
           record_timeout(abort);
           ok = false;
           break;
@@ -581,8 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.wfull[s]);
-        if (++s == SL) {
+        if (lane == 0) ptx::mbar_arrive(&sh.xfull[s]);
+        if (++s == SX) {
           s = 0;
           ph ^= 1;
         }
@@ -759,13 +798,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- teardown: drain what this CTA issued, then free TMEM ----
   if (warp == 0 && lane == 0 && *abort) {
     int no_abort = 0;  // only the last issue to each slot can still be in flight
-    for (int i = 0; i < SL; ++i) {
+    for (int i = 0; i < SW; ++i) {
       if ((wmask >> i) & 1)
         ptx::mbar_wait_bounded(&sh.wfull[i], (wpar >> i) & 1, kDrainLimit, &no_abort);
     }
     for (int i = 0; i < sc_bufs; ++i)
       if ((smask >> i) & 1)
         ptx::mbar_wait_bounded(&sh.sfull[i], (spar >> i) & 1, kDrainLimit, &no_abort);
+  }
+  if (warp == 2 && lane == 0 && *abort) {
+    int no_abort = 0;
+    for (int i = 0; i < SX; ++i) {
+      if ((xmask >> i) & 1)
+        ptx::mbar_wait_bounded(&sh.xfull[i], (xpar >> i) & 1, kDrainLimit, &no_abort);
+    }
   }
   if (warp == 1 && lane == 0 && mma_issued) {
     int no_abort = 0;
@@ -855,23 +901,29 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
   if (attr_err != cudaSuccess) return WOQ_ECUDA;
 
   // The whole scale tile [BN, K/32] of an output tile comes by TMA when its rows are 16-byte
-  // multiples and it is small; otherwise each dequantiser loads its own scales. Two scale
-  // buffers (the next tile's loads overlap the current tile) when shared memory still
-  // leaves at least four load stages, else one.
+  // multiples and it is small; otherwise each dequantiser loads its own scales. Ring depths:
+  // the first (X stages, raw stages) pair below that fits, with two scale buffers (the next
+  // tile's scales load during this one) if they fit too. Four X stages cover the X copy
+  // latency behind the MMAs; four or more raw stages (4 or 8 KB each) keep the dequantisers
+  // ahead of the copy latency.
   const int64_t spr = w.k / 32;
   const bool sc_tma = spr % 8 == 0 && spr <= kTmaScaleCols;
   const int sc_bytes = sc_tma ? static_cast<int>((BN * spr * 2 + 127) & ~int64_t(127)) : 0;
-  const int stage = kAStage + BN * BK * BITS / 8;
-  auto stages_for = [&](int bufs) {
-    return std::min(kMaxSL,
-                    (kSmemMax - make_layout(BITS, BN, kAStage, kBSlot, kSB, 0, sc_bytes, bufs).total) /
-                        stage);
-  };
-  int sc_bufs = sc_tma ? 2 : 1;
-  if (sc_tma && stages_for(2) < 4) sc_bufs = 1;
-  const int sl = stages_for(sc_bufs);
-  if (sl < 2) return WOQ_ESHAPE;
-  const int smem = make_layout(BITS, BN, kAStage, kBSlot, kSB, sl, sc_bytes, sc_bufs).total;
+  constexpr int kDepths[][2] = {{4, 8}, {4, 6}, {3, 8}, {3, 6}, {4, 4}, {3, 4}, {2, 8},
+                                {2, 6}, {2, 4}, {4, 2}, {3, 2}, {2, 2}};
+  int sx = 0, sw = 0, sc_bufs = 1;
+  for (const auto &d : kDepths) {
+    for (int bufs = sc_tma ? 2 : 1; bufs >= 1 && sx == 0; --bufs) {
+      if (make_layout(BITS, BN, kAStage, kBSlot, kSB, d[0], d[1], sc_bytes, bufs).total <= kSmemMax) {
+        sx = d[0];
+        sw = d[1];
+        sc_bufs = bufs;
+      }
+    }
+    if (sx) break;
+  }
+  if (sx < 2) return WOQ_ESHAPE;
+  const int smem = make_layout(BITS, BN, kAStage, kBSlot, kSB, sx, sw, sc_bytes, sc_bufs).total;
 
   const int64_t num_m = (m + TM - 1) / TM;
   CUtensorMap tm_x, tm_w, tm_s;
@@ -917,7 +969,7 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
       cfg.numAttrs = 2;
     }
     if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_s, w.scales, Y, static_cast<int>(m),
-                           static_cast<int>(w.n), static_cast<int>(w.k), sl, sc_bytes, sc_bufs,
+                           static_cast<int>(w.n), static_cast<int>(w.k), sx, sw, sc_bytes, sc_bufs,
                            plan.splits, static_cast<float *>(nullptr), X, lim, stuck) != cudaSuccess)
       return WOQ_ECUDA;
     count_launches(1);
@@ -951,7 +1003,7 @@ int launch_tc(const float *X, int64_t m, const woq_weight &w, float *Y, void *wo
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_s, w.scales, Y, static_cast<int>(m),
-                           static_cast<int>(w.n), static_cast<int>(w.k), sl, sc_bytes, sc_bufs,
+                           static_cast<int>(w.n), static_cast<int>(w.k), sx, sw, sc_bytes, sc_bufs,
                            plan.splits, partials, static_cast<const float *>(nullptr), lim,
                            stuck) != cudaSuccess)
       return WOQ_ECUDA;
