@@ -470,6 +470,37 @@ def run_prefill(layers, groups, device, m: int, reps: int, peaks, peak_kind, wor
             "launches_per_pass": int(per_step)}
 
 
+def run_batched_decode(layers, groups, device, m: int, steps: int, peaks, peak_kind, world):
+    """Batched decode: m activation rows through every fused projection of every block via
+    qgemm's automatic path (the FP32-accurate split tensor-core GEMM for 24 <= m < 128, the
+    CUDA-core kernel below), replayed from CUDA graphs like the M = 1 decode."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    xs = [workloads.activations(m, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
+          for _, mem in groups]
+    ys = [torch.empty(m, group_shape(mem)[0], device=device) for _, mem in groups]
+    need = max(woq.qgemm_workspace_bytes(m, w, "auto") for w in layers[0])
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+
+    def step(i):
+        for g, w in enumerate(layers[i]):
+            woq.qgemm(xs[g], w, path="auto", out=ys[g], workspace=ws)
+
+    stream = torch.cuda.Stream(device)
+    ms, per_step = time_graph_steps(step, len(layers), steps, max(3, steps // 10), stream, world)
+    us_block = ms * 1e3 / steps
+    step_bytes = decode_step_bytes(layers[0])
+    flops = 2.0 * m * sum(n * k for _, n, k in workloads.DECODER_PROJ)
+    path = "split_tc" if 24 <= m < 128 else ("bf16_tc" if m >= 128 else "fp32")
+    return {"workload": f"decoder_block_m{m}", "m": m, "qgemm_path": path,
+            "blocks_timed": steps, "us_per_block": round(us_block, 2),
+            "tokens_per_s": round(m * 1e6 / (us_block * len(layers)), 1),
+            "weight_gbs": round(step_bytes / (us_block * 1e-6) / 1e9, 1),
+            "hbm_frac": round(step_bytes / (us_block * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "algorithmic_tflops": round(flops / (us_block * 1e-6) / 1e12, 2),
+            "peak_source": peak_kind, "launches_per_block": int(per_step)}
+
+
 # --------------------------------------------------------------------------------------
 # CPU oracle (cpu_baseline leg and the reference arm)
 # --------------------------------------------------------------------------------------
@@ -601,6 +632,8 @@ def main(argv=None):
     ap.add_argument("--unfused", action="store_true", help="7 launches per block instead of 4")
     ap.add_argument("--m", type=int, default=1, help="activation rows per decode step (1..64)")
     ap.add_argument("--no-lm-head", action="store_true")
+    ap.add_argument("--batched-m", type=int, default=64,
+                    help="rows of the batched-decode leg (qgemm auto path); <= 1 skips it")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -623,6 +656,9 @@ def main(argv=None):
     if not args.no_prefill:
         out["prefill"] = run_prefill(layers, groups, device, args.prefill_m, 3, peaks, peak_kind,
                                      world)
+    if args.batched_m > 1:
+        out["batched_decode"] = run_batched_decode(layers, groups, device, args.batched_m,
+                                                   280, peaks, peak_kind, world)
     if rank == 0 and not args.no_cpu_baseline and args.m == 1:
         cb, parity = cpu_baseline_leg(layers[0], groups, xs, args.cpu_budget)
         out["cpu_baseline"] = cb
