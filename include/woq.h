@@ -139,9 +139,28 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
  *   x  device, [m, k] float32 row-major, 16-byte aligned, 1 <= m <= 64
  *   w  host pointer to the weight descriptor; n even (rows interleaved as above)
  *   y  device, [m, n/2] float32 row-major; fully overwritten
- * Limits: k <= 8192. Errors: as qgemv, and WOQ_ESHAPE for an odd n.
+ * Limits: k <= 8192; k <= 4096 always fits, larger k while a stage of 16 weight rows and the
+ * x rows of a CTA fit in the kernel's shared-memory budget (int4 up to 7168), else
+ * WOQ_ESHAPE. Errors: as qgemv, and WOQ_ESHAPE for an odd n.
  */
 int qgemv_swiglu(const float *x, int64_t m, const woq_weight *w, float *y, void *stream);
+
+/*
+ * qgemv_residual -- a decode projection with the residual add fused: y[j, i] = (x . W_hat^T)[j, i]
+ * + r[j, i], one FP32 add after the projection, which is computed exactly as qgemv's CUDA-core
+ * form computes it. In a Qwen3-style decoder block the attention output projection and the
+ * MLP down projection each add their result to the residual stream; with r == y the call
+ * updates that stream in place (hidden += o_proj(attn)).
+ *   x  device, [m, k] float32 row-major, 16-byte aligned, 1 <= m <= 64
+ *   w  host pointer to the weight descriptor (read during the call only)
+ *   r  device, [m, n] float32 row-major, 4-byte aligned; may be y itself
+ *   y  device, [m, n] float32 row-major, 4-byte aligned; fully overwritten
+ * Limits: k <= 8192; k <= 4096 always fits, larger k while one stage of weight rows and the
+ * x rows of a CTA fit in the kernel's shared-memory budget (int4 up to 8192, int8 up to 7680),
+ * else WOQ_ESHAPE. Errors: as qgemv, and WOQ_EINVAL if r and y overlap without being equal.
+ */
+int qgemv_residual(const float *x, int64_t m, const woq_weight *w, const float *r, float *y,
+                   void *stream);
 
 /*
  * qgemv_argmax -- greedy pick over a GEMV's outputs without writing them: for each activation
@@ -154,8 +173,10 @@ int qgemv_swiglu(const float *x, int64_t m, const woq_weight *w, float *y, void 
  *   w    host pointer to the weight descriptor (read during the call only)
  *   idx  device, [m] int64, 8-byte aligned; used as scratch during the call, then the index
  *   val  device, [m] float32; the maximum
- * Limits: k <= 8192 and n < 2^31. Errors: as qgemv, and WOQ_ESHAPE for shapes the fused
- * kernel does not cover.
+ * Limits: k <= 8192 and n < 2^31; k <= 4096 always fits, larger k while one stage of weight
+ * rows and the x rows of a CTA fit in the kernel's shared-memory budget (int4 up to 8192,
+ * int8 up to 7680). Errors: as qgemv, and WOQ_ESHAPE for shapes the fused kernel does not
+ * cover.
  */
 int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, float *val,
                  void *stream);

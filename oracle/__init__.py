@@ -29,6 +29,7 @@ from .woq_ref import (  # noqa: F401
     greedy_ref,
     silu_ref,
     swiglu_ref,
+    residual_ref,
     qgemv_argmax_ref,
     bf16_round,
 )

@@ -198,6 +198,16 @@ def swiglu_ref(X: np.ndarray, packed: np.ndarray, scale_bits: np.ndarray, bits: 
     return silu_ref(Y[:, 0::2]) * Y[:, 1::2]
 
 
+def residual_ref(X: np.ndarray, packed: np.ndarray, scale_bits: np.ndarray, bits: int,
+                 R: np.ndarray) -> np.ndarray:
+    """A projection added to the residual stream: qgemv_ref(X, ...) + R in float64. The text
+    backbone is a Qwen3-0.6B-style causal decoder (evermx article on MOSS-Transcribe-Diarize,
+    "Architecture"; LiteRT model card, "Files": Qwen3-0.6B blocks), a pre-norm transformer
+    whose attention output projection and MLP down projection are each added to the hidden
+    state they were computed from."""
+    return qgemv_ref(X, packed, scale_bits, bits) + np.asarray(R, dtype=np.float64)
+
+
 def greedy_ref(Y: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """Greedy decoding's pick over each row of outputs Y [M, N]: the first index of the
     row maximum, and that maximum ("MOSS Transcribe Diarize 0.9B", soniqo Russian guide,

@@ -80,6 +80,16 @@ def test_argument_checks_return_before_touching_a_device():
     assert L.qgemv_argmax(ok_ptr, 1, ctypes.byref(w), ok_ptr + 4, ok_ptr, None) == _lib.WOQ_EALIGN
     wide = _w(k=16384, packed=ok_ptr, scales=ok_ptr)
     assert L.qgemv_argmax(ok_ptr, 1, ctypes.byref(wide), ok_ptr, ok_ptr, None) == _lib.WOQ_ESHAPE
+    # qgemv_residual: 1 <= m <= 64, k <= 8192, r may equal y but not overlap it otherwise
+    R = L.qgemv_residual
+    assert R(ok_ptr, 0, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EINVAL
+    assert R(ok_ptr, 65, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EINVAL
+    assert R(ok_ptr, 1, ctypes.byref(w), None, ok_ptr, None) == _lib.WOQ_EINVAL
+    assert R(ok_ptr, 1, ctypes.byref(w), ok_ptr, None, None) == _lib.WOQ_EINVAL
+    assert R(ok_ptr, 2, ctypes.byref(w), ok_ptr, ok_ptr + 4 * 64, None) == _lib.WOQ_EINVAL  # row 1 of r is row 0 of y
+    assert R(ok_ptr, 1, ctypes.byref(wide), ok_ptr, ok_ptr, None) == _lib.WOQ_ESHAPE
+    assert R(ok_ptr + 4, 1, ctypes.byref(w), ok_ptr, ok_ptr, None) == _lib.WOQ_EALIGN
+    assert R(ok_ptr, 1, ctypes.byref(w), ok_ptr + 2, ok_ptr + 2, None) == _lib.WOQ_EALIGN
     # bf16 path: workspace checked before the device
     need = L.qgemm_workspace_bytes(256, ctypes.byref(w), _lib.WOQ_PATH_BF16_TC)
     assert need == 256 * 64 * 2

@@ -415,3 +415,20 @@ def test_swiglu_ref_pairs_gate_and_up_rows():
     g, u = 7.0 * 8.0, 7.0 * 2.0
     assert y[0, 1] == pytest.approx(oracle.silu_ref(np.array(g))[()] * u, rel=1e-15)
     assert y[0, 1] == pytest.approx(g * u, rel=1e-20)  # sigmoid(56) is 1 to double precision
+
+
+def test_residual_ref_adds_the_projection_to_the_stream():
+    # W = 0 leaves the stream as it is; a one-hot weight row adds one x column, exactly
+    K = 64
+    rng = np.random.default_rng(3)
+    R = rng.standard_normal((3, 5))
+    X = rng.standard_normal((3, K)).astype(np.float32)
+    q, s = oracle.quantise(np.zeros((5, K), dtype=np.float32), 4)
+    assert np.array_equal(oracle.residual_ref(X, oracle.pack(q, 4), s, 4, R), R)
+    W = np.zeros((5, K), dtype=np.float32)
+    W[2, 7] = 7.0  # block max 7 -> scale 1, code 7
+    q, s = oracle.quantise(W, 4)
+    Y = oracle.residual_ref(X, oracle.pack(q, 4), s, 4, R)
+    want = R.copy()
+    want[:, 2] += 7.0 * X[:, 7].astype(np.float64)
+    assert np.array_equal(Y, want)

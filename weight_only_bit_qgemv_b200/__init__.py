@@ -36,6 +36,7 @@ __all__ = [
     "qgemv",
     "qgemv_argmax",
     "qgemv_swiglu",
+    "qgemv_residual",
     "interleave_rows",
     "qgemm",
     "qgemm_workspace_bytes",
@@ -158,6 +159,23 @@ def qgemv_argmax(x: torch.Tensor, w: PackedWeight, stream=None) -> tuple[torch.T
     rc = _lib.lib().qgemv_argmax(_ptr(x), m, ctypes.byref(d), _ptr(idx), _ptr(val), _stream(stream))
     _lib.check(rc, "qgemv_argmax")
     return idx, val
+
+
+def qgemv_residual(x: torch.Tensor, w: PackedWeight, r: torch.Tensor, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """y = x . W_hat^T + r with the add fused (C ABI ``qgemv_residual``); ``out`` may be ``r``
+    for an in-place update of the residual stream."""
+    if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
+    m = x.shape[0]
+    if r.dtype != torch.float32 or not r.is_cuda or tuple(r.shape) != (m, w.n) or not r.is_contiguous():
+        raise ValueError("r must be a contiguous float32 CUDA tensor of shape [m, n]")
+    if out is None:
+        out = torch.empty(m, w.n, dtype=torch.float32, device=x.device)
+    d = w.desc()
+    rc = _lib.lib().qgemv_residual(_ptr(x), m, ctypes.byref(d), _ptr(r), _ptr(out), _stream(stream))
+    _lib.check(rc, "qgemv_residual")
+    return out
 
 
 def qgemm_workspace_bytes(m: int, w: PackedWeight, path: str = "auto") -> int:

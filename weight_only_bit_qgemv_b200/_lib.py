@@ -32,6 +32,7 @@ EXPORTS = (
     "qgemv",
     "qgemv_path",
     "qgemv_swiglu",
+    "qgemv_residual",
     "qgemv_argmax",
     "qgemm_workspace_bytes",
     "qgemm",
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
     L.qgemv_path.restype = ctypes.c_int
     L.qgemv_swiglu.argtypes = [vp, c_i64, wp, vp, vp]
     L.qgemv_swiglu.restype = ctypes.c_int
+    L.qgemv_residual.argtypes = [vp, c_i64, wp, vp, vp, vp]
+    L.qgemv_residual.restype = ctypes.c_int
     L.qgemv_argmax.argtypes = [vp, c_i64, wp, vp, vp, vp]
     L.qgemv_argmax.restype = ctypes.c_int
     L.qgemm_workspace_bytes.argtypes = [c_i64, wp, c_i32]

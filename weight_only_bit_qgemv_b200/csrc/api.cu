@@ -112,6 +112,24 @@ int qgemv_swiglu(const float *x, int64_t m, const woq_weight *w, float *y, void 
   return woq::launch_gemv_swiglu(x, m, *w, y, static_cast<cudaStream_t>(stream), dev);
 }
 
+int qgemv_residual(const float *x, int64_t m, const woq_weight *w, const float *r, float *y,
+                   void *stream) {
+  int rc = woq::check_weight(w);
+  if (rc != WOQ_OK) return rc;
+  if (!x || !r || !y) return WOQ_EINVAL;
+  if (m < 1 || m > 64) return WOQ_EINVAL;
+  if (w->k > 8192) return WOQ_ESHAPE;
+  // r may be y itself; any other overlap of the two [m, n] arrays is refused
+  const uintptr_t rb = reinterpret_cast<uintptr_t>(r), yb = reinterpret_cast<uintptr_t>(y);
+  const uintptr_t bytes = static_cast<uintptr_t>(m) * static_cast<uintptr_t>(w->n) * sizeof(float);
+  if (rb != yb && rb < yb + bytes && yb < rb + bytes) return WOQ_EINVAL;
+  if (!woq::aligned(x, 16) || !woq::aligned(r, 4) || !woq::aligned(y, 4)) return WOQ_EALIGN;
+  DevInfo dev;
+  rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  return woq::launch_gemv_residual(x, m, *w, r, y, static_cast<cudaStream_t>(stream), dev);
+}
+
 int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, float *val,
                  void *stream) {
   int rc = woq::check_weight(w);

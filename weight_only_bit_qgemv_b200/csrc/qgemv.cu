@@ -465,8 +465,10 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int row) {
 // Epilogues. kEpiWrite: y[m, n] is written. kEpiArgmax: nothing is written to y; for each
 // activation row the CTA's largest key over its outputs goes into keys[row] by a 64-bit
 // atomicMax. kEpiSwiglu: rows 2i and 2i+1 are a gate and an up projection (RW even, so a
-// warp holds both); y[m, n/2] gets silu(gate) * up.
-constexpr int kEpiWrite = 0, kEpiArgmax = 1, kEpiSwiglu = 2;
+// warp holds both); y[m, n/2] gets silu(gate) * up. kEpiResidual: y[m, n] = the output +
+// resid[m, n], one FP32 add (resid may be y itself: each element is read, then written, by
+// the one lane that owns it).
+constexpr int kEpiWrite = 0, kEpiArgmax = 1, kEpiSwiglu = 2, kEpiResidual = 3;
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
                      const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n,
                      int k, int stages, int stage_bytes, int x_bytes,
-                     unsigned long long *__restrict__ keys = nullptr) {
+                     unsigned long long *__restrict__ keys = nullptr, const float *resid = nullptr) {
   constexpr int kBulkWarps = NW;
   constexpr int TR = kBulkWarps * RW;
   constexpr bool AMAX = EPI == kEpiArgmax;
@@ -617,6 +619,9 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
           if constexpr (AMAX) {
             const unsigned long long key = argmax_key(acc[r][mm], row0 + r);
             best = key > best ? key : best;
+          } else if constexpr (EPI == kEpiResidual) {
+            const size_t o = static_cast<size_t>(m0 + mm) * n + row0 + r;
+            y[o] = acc[r][mm] + resid[o];
           } else if constexpr (EPI == kEpiSwiglu) {
             // every lane holds every row's sum after the butterfly: the up row r + 1 is here
             if (r % 2 == 0)
@@ -754,7 +759,7 @@ constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
 template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
 int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                   const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes,
-                  unsigned long long *keys = nullptr) {
+                  unsigned long long *keys = nullptr, const float *resid = nullptr) {
   auto kern = gemv_bulk_kernel<BITS, MT, RW, NW, EPI>;
   constexpr int kBulkThreads = bulk_threads(NW);
   constexpr int TR = NW * RW;
@@ -786,7 +791,7 @@ int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cuda
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, w.packed, w.scales, y, static_cast<int>(m),
                                            static_cast<int>(w.n), static_cast<int>(w.k),
                                            static_cast<int>(stages), static_cast<int>(stage_bytes),
-                                           static_cast<int>(x_bytes), keys);
+                                           static_cast<int>(x_bytes), keys, resid);
   if (e != cudaSuccess) return WOQ_ECUDA;
   count_launches(1);
   return WOQ_OK;
@@ -802,7 +807,7 @@ inline int bulk_rows_per_warp(int nw, int rw_max, size_t row_total) {
 template <int BITS, int MT, int NW, int EPI = kEpiWrite>
 int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                    const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes,
-                   unsigned long long *keys = nullptr) {
+                   unsigned long long *keys = nullptr, const float *resid = nullptr) {
   // More rows per warp only where registers allow.
   int rw = bulk_rows_per_warp(NW, NW == 16 ? 2 : MT <= 2 ? 4 : 2, row_total);
   const size_t stage_bytes = (static_cast<size_t>(NW) * rw * row_total + 127) & ~size_t(127);
@@ -810,15 +815,17 @@ int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cud
   if (w.n < NW * rw) rw = 1;  // tiny n: one row per warp, all from global memory
   if constexpr (MT <= 2 && NW == 8) {
     if (rw == 4)
-      return launch_bulk_t<BITS, MT, 4, NW, EPI>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
+      return launch_bulk_t<BITS, MT, 4, NW, EPI>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys,
+                                                 resid);
   }
   if constexpr (NW == 8 || MT == 1) {
     if (rw >= 2)
-      return launch_bulk_t<BITS, MT, 2, NW, EPI>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys);
+      return launch_bulk_t<BITS, MT, 2, NW, EPI>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys,
+                                                 resid);
   }
   return launch_bulk_t<BITS, MT, 1, NW, EPI>(x, m, w, y, s, dev, pdl,
                                               (static_cast<size_t>(NW) * row_total + 127) & ~size_t(127),
-                                              x_bytes, keys);
+                                              x_bytes, keys, resid);
 }
 
 template <int BITS, int MT>
@@ -883,6 +890,19 @@ __global__ void __launch_bounds__(32) argmax_final_kernel(unsigned long long *ke
       static_cast<long long>(0xFFFFFFFFu - static_cast<uint32_t>(key & 0xFFFFFFFFull));
 }
 
+// Calls go(MT) for x-row tiles of MT = the smallest of 1, 2, 4, 8 that covers m, then for
+// smaller MT while the launch does not fit in a CTA's shared memory (go returns 1): fewer x
+// rows per CTA leave room for longer rows. Returns 1 if not even MT = 1 fits.
+template <typename Go>
+int with_fitting_mt(int64_t m, Go &&go) {
+  const int want = m == 1 ? 1 : m == 2 ? 2 : m <= 4 ? 4 : 8;
+  int rc = 1;
+  if (want >= 8 && (rc = go(std::integral_constant<int, 8>())) != 1) return rc;
+  if (want >= 4 && (rc = go(std::integral_constant<int, 4>())) != 1) return rc;
+  if (want >= 2 && (rc = go(std::integral_constant<int, 2>())) != 1) return rc;
+  return go(std::integral_constant<int, 1>());
+}
+
 // qgemv_swiglu: the bulk GEMV with two rows (gate, up) per warp.
 template <int BITS>
 int swiglu_bulk(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
@@ -893,35 +913,54 @@ int swiglu_bulk(const float *x, int64_t m, const woq_weight &w, float *y, cudaSt
     constexpr int NW = decltype(nw_tag)::value;
     const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
     const size_t stage_bytes = (static_cast<size_t>(NW) * 2 * row_total + 127) & ~size_t(127);
-    if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return WOQ_ESHAPE;
+    if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return 1;
     return launch_bulk_t<BITS, MT, 2, NW, kEpiSwiglu>(x, m, w, y, s, dev, true, stage_bytes, x_bytes);
   };
-  using I1 = std::integral_constant<int, 1>;
   using I8 = std::integral_constant<int, 8>;
   using I16 = std::integral_constant<int, 16>;
-  if (m == 1) {
-    // as qgemv: 16 warps while each CTA gets at most two tiles
-    if (w.n / 32 <= 2 * static_cast<int64_t>(dev.sm_count)) return go(I1(), I16());
-    return go(I1(), I8());
-  }
-  if (m == 2) return go(std::integral_constant<int, 2>(), I8());
-  if (m <= 4) return go(std::integral_constant<int, 4>(), I8());
-  return go(I8(), I8());
+  return with_fitting_mt(m, [&](auto mt_tag) -> int {
+    if constexpr (decltype(mt_tag)::value == 1) {
+      // as qgemv: 16 warps while each CTA gets at most two tiles
+      if (w.n / 32 <= 2 * static_cast<int64_t>(dev.sm_count)) {
+        const int rc = go(mt_tag, I16());
+        if (rc != 1) return rc;
+      }
+    }
+    return go(mt_tag, I8());
+  });
 }
 
 template <int BITS>
 int argmax_bulk(const float *x, int64_t m, const woq_weight &w, unsigned long long *keys,
                 cudaStream_t s, const DevInfo &dev) {
   const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
-  auto go = [&](auto mt_tag) -> int {
+  return with_fitting_mt(m, [&](auto mt_tag) -> int {
     constexpr int MT = decltype(mt_tag)::value;
     const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
     return launch_bulk_nw<BITS, MT, 8, kEpiArgmax>(x, m, w, nullptr, s, dev, true, row_total, x_bytes, keys);
-  };
-  if (m == 1) return go(std::integral_constant<int, 1>());
-  if (m == 2) return go(std::integral_constant<int, 2>());
-  if (m <= 4) return go(std::integral_constant<int, 4>());
-  return go(std::integral_constant<int, 8>());
+  });
+}
+
+// qgemv_residual: the bulk GEMV (row and warp choices as qgemv's) with the residual add.
+template <int BITS>
+int residual_bulk(const float *x, int64_t m, const woq_weight &w, const float *r, float *y,
+                  cudaStream_t s, const DevInfo &dev) {
+  const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
+  return with_fitting_mt(m, [&](auto mt_tag) -> int {
+    constexpr int MT = decltype(mt_tag)::value;
+    const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
+    if constexpr (MT == 1) {
+      const int rw16 = bulk_rows_per_warp(16, 2, row_total);
+      const int64_t tiles16 = w.n / (16 * rw16);
+      if (tiles16 >= 1 && tiles16 <= 2 * static_cast<int64_t>(dev.sm_count)) {
+        const int rc = launch_bulk_nw<BITS, MT, 16, kEpiResidual>(x, m, w, y, s, dev, true, row_total,
+                                                                  x_bytes, nullptr, r);
+        if (rc != 1) return rc;
+      }
+    }
+    return launch_bulk_nw<BITS, MT, 8, kEpiResidual>(x, m, w, y, s, dev, true, row_total, x_bytes,
+                                                     nullptr, r);
+  });
 }
 
 }  // namespace
@@ -944,7 +983,15 @@ int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, c
 
 int launch_gemv_swiglu(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                        const DevInfo &dev) {
-  return w.bits == 4 ? swiglu_bulk<4>(x, m, w, y, s, dev) : swiglu_bulk<8>(x, m, w, y, s, dev);
+  const int rc = w.bits == 4 ? swiglu_bulk<4>(x, m, w, y, s, dev) : swiglu_bulk<8>(x, m, w, y, s, dev);
+  return rc == 1 ? WOQ_ESHAPE : rc;
+}
+
+int launch_gemv_residual(const float *x, int64_t m, const woq_weight &w, const float *r, float *y,
+                         cudaStream_t s, const DevInfo &dev) {
+  const int rc = w.bits == 4 ? residual_bulk<4>(x, m, w, r, y, s, dev)
+                             : residual_bulk<8>(x, m, w, r, y, s, dev);
+  return rc == 1 ? WOQ_ESHAPE : rc;
 }
 
 int launch_gemv_argmax(const float *x, int64_t m, const woq_weight &w, int64_t *idx, float *val,

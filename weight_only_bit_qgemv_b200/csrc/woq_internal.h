@@ -39,6 +39,9 @@ int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, c
 // qgemv_swiglu: y[m, n/2] = silu(rows 2i) * rows 2i+1 of x . W_hat^T.
 int launch_gemv_swiglu(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                        const DevInfo &dev);
+// qgemv_residual: y[m, n] = x . W_hat^T + r (r may be y).
+int launch_gemv_residual(const float *x, int64_t m, const woq_weight &w, const float *r, float *y,
+                         cudaStream_t s, const DevInfo &dev);
 // qgemv_argmax: zero the keys in idx, the argmax GEMV, then keys -> (idx, val).
 int launch_gemv_argmax(const float *x, int64_t m, const woq_weight &w, int64_t *idx, float *val,
                        cudaStream_t s, const DevInfo &dev);
