@@ -501,6 +501,50 @@ def run_batched_decode(layers, groups, device, m: int, steps: int, peaks, peak_k
             "peak_source": peak_kind, "launches_per_block": int(per_step)}
 
 
+def run_fused_epilogues(layers, groups, device, steps: int, peaks, world):
+    """The decode-step projections whose neighbours fuse (NEXT-4 rows): gate|up with the SwiGLU
+    (qgemv_swiglu, the gate|up outputs never written) and down with the residual add
+    (qgemv_residual, in place on the hidden state), each against the plain qgemv of the same
+    weights; M = 1, all 28 blocks cycled, CUDA graphs as the decode steps. Timing only: the
+    decode step's gate|up matrix is packed as gate rows then up rows, not interleaved, which
+    changes which rows pair up but not the work."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    names = [nm for nm, _ in groups]
+    if "gate_up" not in names or "down" not in names:
+        return None
+    gu, dn = names.index("gate_up"), names.index("down")
+    n_gu, k_gu = group_shape(groups[gu][1])
+    n_dn, k_dn = group_shape(groups[dn][1])
+    x_gu = workloads.activations(1, k_gu, seed=11).to(device)
+    x_dn = workloads.activations(1, k_dn, seed=12).to(device)
+    y_gu = torch.empty(1, n_gu, device=device)
+    y_sw = torch.empty(1, n_gu // 2, device=device)
+    h = torch.zeros(1, n_dn, device=device)
+    y_dn = torch.empty(1, n_dn, device=device)
+    stream = torch.cuda.Stream(device)
+    warm = max(3, steps // 10)
+
+    def timed(fn):
+        ms, per_step = time_graph_steps(fn, len(layers), steps, warm, stream, world)
+        return ms * 1e3 / steps, int(per_step)
+
+    out = {"m": 1, "calls_timed": steps}
+    for key, plain, fused, idx in (
+        ("swiglu_gate_up", lambda i: woq.qgemv(x_gu, layers[i][gu], out=y_gu),
+         lambda i: woq.qgemv_swiglu(x_gu, layers[i][gu], out=y_sw), gu),
+        ("residual_down", lambda i: woq.qgemv(x_dn, layers[i][dn], out=y_dn),
+         lambda i: woq.qgemv_residual(x_dn, layers[i][dn], h, out=h), dn),
+    ):
+        nbytes = layers[0][idx].nbytes
+        us_plain, _ = timed(plain)
+        us_fused, launches = timed(fused)
+        out[key] = {"shape": f"[{layers[0][idx].n}x{layers[0][idx].k}]", "us_per_call": round(us_fused, 3),
+                    "plain_qgemv_us": round(us_plain, 3), "launches_per_call": launches,
+                    "weight_gbs": round(nbytes / (us_fused * 1e-6) / 1e9, 1)}
+    return out
+
+
 # --------------------------------------------------------------------------------------
 # CPU oracle (cpu_baseline leg and the reference arm)
 # --------------------------------------------------------------------------------------
@@ -632,6 +676,7 @@ def main(argv=None):
     ap.add_argument("--unfused", action="store_true", help="7 launches per block instead of 4")
     ap.add_argument("--m", type=int, default=1, help="activation rows per decode step (1..64)")
     ap.add_argument("--no-lm-head", action="store_true")
+    ap.add_argument("--no-fused-epilogues", action="store_true")
     ap.add_argument("--batched-m", type=int, default=64,
                     help="rows of the batched-decode leg (qgemm auto path); <= 1 skips it")
     args = ap.parse_args(argv)
@@ -659,6 +704,10 @@ def main(argv=None):
     if args.batched_m > 1:
         out["batched_decode"] = run_batched_decode(layers, groups, device, args.batched_m,
                                                    280, peaks, peak_kind, world)
+    if not args.no_fused_epilogues:
+        fe = run_fused_epilogues(layers, groups, device, 2800, peaks, world)
+        if fe is not None:
+            out["fused_epilogues"] = fe
     if rank == 0 and not args.no_cpu_baseline and args.m == 1:
         cb, parity = cpu_baseline_leg(layers[0], groups, xs, args.cpu_budget)
         out["cpu_baseline"] = cb

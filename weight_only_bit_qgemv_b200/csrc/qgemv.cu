@@ -580,6 +580,14 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     const uint8_t *stage = ring + static_cast<size_t>(s) * stage_bytes;
     const int lrow0 = warp * RW;  // this warp's first row within the tile
     const int row0 = tile * TR + lrow0;
+    // Residual mode: the lane that will store output (row0 + lane / MT, x row lane % MT)
+    // fetches its residual now, so that the load's latency hides behind the dot products.
+    float res = 0.f;
+    if constexpr (EPI == kEpiResidual) {
+      const int rr = lane / MT, mm = lane % MT;
+      if (rr < RW && row0 + rr < n && m0 + mm < m)
+        res = resid[static_cast<size_t>(m0 + mm) * n + row0 + rr];
+    }
     float acc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
@@ -620,8 +628,7 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
             const unsigned long long key = argmax_key(acc[r][mm], row0 + r);
             best = key > best ? key : best;
           } else if constexpr (EPI == kEpiResidual) {
-            const size_t o = static_cast<size_t>(m0 + mm) * n + row0 + r;
-            y[o] = acc[r][mm] + resid[o];
+            y[static_cast<size_t>(m0 + mm) * n + row0 + r] = acc[r][mm] + res;
           } else if constexpr (EPI == kEpiSwiglu) {
             // every lane holds every row's sum after the butterfly: the up row r + 1 is here
             if (r % 2 == 0)
