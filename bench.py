@@ -501,7 +501,7 @@ def run_batched_decode(layers, groups, device, m: int, steps: int, peaks, peak_k
             "peak_source": peak_kind, "launches_per_block": int(per_step)}
 
 
-def run_fused_epilogues(layers, groups, device, steps: int, peaks, world):
+def run_fused_epilogues(layers, groups, device, steps: int, world):
     """The decode-step projections whose neighbours fuse (NEXT-4 rows): gate|up with the SwiGLU
     (qgemv_swiglu, the gate|up outputs never written) and down with the residual add
     (qgemv_residual, in place on the hidden state), each against the plain qgemv of the same
@@ -705,7 +705,7 @@ def main(argv=None):
         out["batched_decode"] = run_batched_decode(layers, groups, device, args.batched_m,
                                                    280, peaks, peak_kind, world)
     if not args.no_fused_epilogues:
-        fe = run_fused_epilogues(layers, groups, device, 2800, peaks, world)
+        fe = run_fused_epilogues(layers, groups, device, 2800, world)
         if fe is not None:
             out["fused_epilogues"] = fe
     if rank == 0 and not args.no_cpu_baseline and args.m == 1:

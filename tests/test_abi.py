@@ -8,7 +8,6 @@ import ctypes
 import os
 import re
 
-import pytest
 
 from weight_only_bit_qgemv_b200 import _lib
 

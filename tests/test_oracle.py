@@ -8,7 +8,6 @@ order or a transposed operand in the oracle fails at least one of them.
 """
 
 import bisect
-import math
 import struct
 from fractions import Fraction
 
@@ -96,7 +95,7 @@ def test_fp16_round_ties_to_even_at_exact_midpoints():
         assert int(oracle.fp16_round(np.float64(mid))) == want
 
 
-def test_scale_closed_forms(golden_dir):
+def test_scale_closed_forms():
     for row in read_rows("scale_closed_form.txt"):
         bits, a = int(row[0]), float(row[1])
         W = np.zeros((1, 32), dtype=np.float32)

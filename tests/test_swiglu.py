@@ -1,6 +1,5 @@
 """GPU parity of qgemv_swiglu (gate|up GEMV with a fused SwiGLU) against the oracle."""
 
-import numpy as np
 import pytest
 import torch
 
