@@ -100,10 +100,12 @@ int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, u
 /*
  * qgemv -- decode path, y[m, n] = x[m, k] . W_hat^T for 1 <= m <= 64 ("TinyMOSS-Diarize",
  * "How we built it": the separate GEMV path for decode). FP32 accuracy: within a 32-block
- * the codes are multiplied exactly and the block sum is scaled once, in FP32. Small batches
- * (m >= 8) over wide matrices (n / 128 >= SM count) take the tensor-core form of qgemv_path
- * WOQ_GEMV_SPLIT_TC, every other call the CUDA-core form. Deterministic: the same inputs give
- * the same bits on every call.
+ * the codes are multiplied exactly and the block sum is scaled once, in FP32 (CUDA-core and
+ * WOQ_GEMV_SPLIT_TC forms), or x and s*q go to the tcgen05 tensor cores as bf16 hi + lo pairs
+ * (WOQ_GEMV_SPLIT_GEMM). The kernel is chosen by shape, as measured on B200: m >= 24 on
+ * narrow matrices and m >= 48 on wide ones (n / 128 >= SM count) take WOQ_GEMV_SPLIT_GEMM,
+ * 8 <= m < 48 on wide matrices WOQ_GEMV_SPLIT_TC, every other call the CUDA-core form.
+ * Deterministic: the same inputs give the same bits on every call.
  *   x  device, [m, k] float32 row-major, 16-byte aligned
  *   w  host pointer to the weight descriptor (read during the call only)
  *   y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
@@ -122,11 +124,15 @@ int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream
  *                       scaled by its binary16 scale in FP32. The split keeps 16 of x's 24
  *                       significand bits; error stays within the FP32 tolerance of qgemv.
  *                       Needs 2 <= m <= 64, k % 256 == 0 and k <= 8192, else WOQ_ESHAPE.
+ *   WOQ_GEMV_SPLIT_GEMM the tcgen05 split GEMM of qgemm's WOQ_PATH_SPLIT_TC (x and s*q each
+ *                       as bf16 hi + lo, all four products in an FP32 tensor-memory
+ *                       accumulator, 64-row tiles); no workspace. Any 1 <= m <= 64.
  * Arguments and errors otherwise as qgemv; an unknown path is WOQ_EINVAL.
  */
 #define WOQ_GEMV_AUTO       0
 #define WOQ_GEMV_CUDA_CORE  1
 #define WOQ_GEMV_SPLIT_TC   2
+#define WOQ_GEMV_SPLIT_GEMM 3
 int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t path,
                void *stream);
 

@@ -202,3 +202,27 @@ def test_auto_and_cuda_core_paths_agree_bitwise_on_decoder_shapes():
     a = woq.qgemv(x, w)
     b = woq.qgemv(x, w, path="cuda_core")
     assert torch.equal(a, b), name
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("proj", [0, 3, 6])
+@pytest.mark.parametrize("m", [1, 24, 64])
+def test_split_gemm_path(bits, proj, m):
+    """qgemv through the tcgen05 split GEMM (x and s*q as bf16 hi + lo): FP32 tolerance."""
+    name, n, k = workloads.DECODER_PROJ[proj]
+    W = workloads.weight(n, k, seed=workloads.layer_seed(6, proj))
+    w, p, s = packed_from_weight(W, bits)
+    x = workloads.activations(m, k, seed=m + 3)
+    buf, y = guarded_out(m, n)
+    woq.qgemv(x.cuda(), w, out=y, path="split_gemm")
+    assert tail_intact(buf, m, n)
+    assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL, name
+
+
+def test_auto_routes_batched_decode_to_the_split_gemm():
+    name, n, k = workloads.DECODER_PROJ[6]
+    W = workloads.weight(n, k, seed=7)
+    w, _, _ = packed_from_weight(W, 4)
+    for m, same_as in ((16, "cuda_core"), (24, "split_gemm"), (64, "split_gemm")):
+        x = workloads.activations(m, k, seed=m).cuda()
+        assert torch.equal(woq.qgemv(x, w), woq.qgemv(x, w, path=same_as)), (m, same_as)

@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     WOQ_GEMV_AUTO,
     WOQ_GEMV_CUDA_CORE,
     WOQ_GEMV_SPLIT_TC,
+    WOQ_GEMV_SPLIT_GEMM,
     WOQ_PATH_AUTO,
     WOQ_PATH_BF16_TC,
     WOQ_PATH_FP32,
@@ -51,7 +52,12 @@ _PATHS = {
     "bf16_tc": WOQ_PATH_BF16_TC,
     "split_tc": WOQ_PATH_SPLIT_TC,
 }
-_GEMV_PATHS = {"auto": WOQ_GEMV_AUTO, "cuda_core": WOQ_GEMV_CUDA_CORE, "split_tc": WOQ_GEMV_SPLIT_TC}
+_GEMV_PATHS = {
+    "auto": WOQ_GEMV_AUTO,
+    "cuda_core": WOQ_GEMV_CUDA_CORE,
+    "split_tc": WOQ_GEMV_SPLIT_TC,
+    "split_gemm": WOQ_GEMV_SPLIT_GEMM,
+}
 
 
 def _ptr(t: torch.Tensor) -> int:
@@ -115,7 +121,7 @@ def qgemv(
     path: str = "auto",
 ) -> torch.Tensor:
     """y[m, n] = x[m, k] . W_hat^T, 1 <= m <= 64, FP32 accuracy (C ABI ``qgemv_path``);
-    path in {"auto", "cuda_core", "split_tc"}."""
+    path in {"auto", "cuda_core", "split_tc", "split_gemm"}."""
     if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
         raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
     m = x.shape[0]

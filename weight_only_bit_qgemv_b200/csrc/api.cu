@@ -66,10 +66,13 @@ using woq::DevInfo;
 
 extern "C" {
 
-// qgemv runs on the tensor cores from this many activation rows on, for matrices wide
-// enough that 128-row tiles cover every SM; measured on B200, the CUDA-core kernel is faster
-// for fewer rows and for the narrower decoder projections.
+// qgemv's automatic choice, measured on B200. The tcgen05 split GEMM (no workspace) from
+// kGemmMinM rows on for the decoder projections and from kGemmMinMWide on for matrices wide
+// enough that 128-row tiles cover every SM (the lm_head); the small-batch mma.sync form for
+// the wide ones from kTcMinM rows up to there; the CUDA-core kernel otherwise.
 constexpr int64_t kTcMinM = 8;
+constexpr int64_t kGemmMinM = 24;
+constexpr int64_t kGemmMinMWide = 48;
 
 int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t path,
                void *stream) {
@@ -77,7 +80,8 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
   if (rc != WOQ_OK) return rc;
   if (!x || !y) return WOQ_EINVAL;
   if (m < 1 || m > 64) return WOQ_EINVAL;
-  if (path != WOQ_GEMV_AUTO && path != WOQ_GEMV_CUDA_CORE && path != WOQ_GEMV_SPLIT_TC)
+  if (path != WOQ_GEMV_AUTO && path != WOQ_GEMV_CUDA_CORE && path != WOQ_GEMV_SPLIT_TC &&
+      path != WOQ_GEMV_SPLIT_GEMM)
     return WOQ_EINVAL;
   if (w->k > 32768) return WOQ_ESHAPE;
   if (!woq::aligned(x, 16) || !woq::aligned(y, 16)) return WOQ_EALIGN;
@@ -85,8 +89,13 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
   rc = woq::current_device(&dev);
   if (rc != WOQ_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool tc = path == WOQ_GEMV_SPLIT_TC ||
-                  (path == WOQ_GEMV_AUTO && m >= kTcMinM && (w->n + 127) / 128 >= dev.sm_count);
+  const bool wide = (w->n + 127) / 128 >= dev.sm_count;
+  if (path == WOQ_GEMV_SPLIT_GEMM ||
+      (path == WOQ_GEMV_AUTO && m >= (wide ? kGemmMinMWide : kGemmMinM))) {
+    const woq::GemmPlan plan = woq::plan_gemm_tc(m, w->n, w->k, dev.sm_count, SIZE_MAX, true);
+    return woq::launch_gemm_tc(x, m, *w, y, nullptr, plan, s, dev);
+  }
+  const bool tc = path == WOQ_GEMV_SPLIT_TC || (path == WOQ_GEMV_AUTO && m >= kTcMinM && wide);
   if (tc) {
     rc = woq::launch_gemv_tc(x, m, *w, y, s, dev);
     if (rc != 1) return rc;
