@@ -117,3 +117,15 @@ def test_workspace_sizing():
 
 def test_launch_counter_starts_readable():
     assert _lib.lib().woq_launch_count() >= 0
+
+
+def test_binding_constants_match_the_header():
+    """Every integer #define of include/woq.h has the same value in the Python binding."""
+    import os
+    import re
+
+    header = open(os.path.join(os.path.dirname(_lib.__file__), "..", "include", "woq.h")).read()
+    defines = dict(re.findall(r"^#define (WOQ_\w+)\s+(-?\d+)\b", header, flags=re.M))
+    assert len(defines) >= 17
+    for name, value in defines.items():
+        assert getattr(_lib, name) == int(value), name
