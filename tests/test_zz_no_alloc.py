@@ -57,3 +57,31 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     m_too_big = (32 << 20) // (2 * k) + 1          # bf16 copy of X would exceed 32 MiB
     rc = _lib.lib().qgemm_bf16_noalloc(X.data_ptr(), m_too_big, ctypes.byref(d), Y.data_ptr(), None)
     assert rc == _lib.WOQ_ESHAPE
+
+
+def test_noalloc_allocates_nothing_and_accepts_the_exact_fit():
+    """A call whose bf16 copy of X fills the 32 MiB scratch exactly is accepted and matches the
+    workspace path, and a call (after a first one has loaded the library's kernels) leaves the
+    device's free memory and torch's allocations unchanged."""
+    n, k = 256, 2048
+    W = workloads.weight(n, k, seed=21)
+    w, _, _ = packed_from_weight(W, 4)
+    m = (32 << 20) // (2 * k)                      # m * k * 2 == 32 MiB exactly
+    X = workloads.activations(m, k, seed=22).cuda()
+    Y = torch.full((m, n), float("nan"), device="cuda")
+    assert _noalloc(X, w, Y) == _lib.WOQ_OK       # first call: loads modules, looks up the array
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    Y2 = torch.full((m, n), float("nan"), device="cuda")
+    alloc1 = torch.cuda.memory_allocated()
+    free1, _ = torch.cuda.mem_get_info()
+    assert _noalloc(X, w, Y2) == _lib.WOQ_OK
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free1
+    assert torch.cuda.memory_allocated() == alloc1
+    assert alloc1 - alloc0 == Y2.numel() * 4 and free0 >= free1
+    Y_ref = woq.qgemm(X, w, path="bf16_tc")
+    assert fro_rel(Y2.cpu().numpy(), Y_ref.cpu().numpy()) <= BF16_READING_TOL
+    assert torch.equal(Y, Y2)
+    assert woq.device_status() == _lib.WOQ_OK

@@ -10,12 +10,12 @@
 // That array is a file-scope __device__ symbol of kScratchBytes (32 MiB). Every GPU that
 // loads the library holds it until the process exits. In host code its name is only a
 // host-side stand-in for the symbol, never a device address, so the real address is
-// looked up once per device with cudaGetSymbolAddress (with that device current) and
-// cached. All calls on a device share the one array; its contents after a call are that
+// looked up with cudaGetSymbolAddress (with that device current) on a device's first call
+// and cached once the lookup has succeeded. All calls on a device share the one array; its contents after a call are that
 // call's bf16 copy of X, and every call overwrites the part it reads before reading it, so
 // nothing has to be cleared. Two calls whose kernels overlap on the GPU (for example on two
 // streams without ordering between them) race on the array.
-#include <mutex>
+#include <atomic>
 
 #include "woq.h"
 #include "woq_internal.h"
@@ -28,21 +28,23 @@ constexpr size_t kScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void *g_ptr[kMaxDevices];
-int g_rc[kMaxDevices];
+std::atomic<void *> g_ptr[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array on the current device. Only a successful lookup is
+// cached: a failed one (for example a first call made while a stream is being captured)
+// fails that call alone, and the next call looks the address up again.
 int scratch_address(int device, void **out) {
   if (device < 0 || device >= kMaxDevices) return WOQ_EDEVICE;
-  std::call_once(g_once[device], [device] {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_ptr[device] = p;
-    g_rc[device] = (e == cudaSuccess && p != nullptr) ? WOQ_OK : WOQ_ECUDA;
-  });
-  *out = g_ptr[device];
-  return g_rc[device];
+  void *p = g_ptr[device].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();  // reset the runtime's last-error state, which the lookup set
+      return WOQ_ECUDA;
+    }
+    g_ptr[device].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return WOQ_OK;
 }
 
 }  // namespace

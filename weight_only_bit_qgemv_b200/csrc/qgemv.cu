@@ -472,10 +472,11 @@ constexpr int kEpiWrite = 0, kEpiArgmax = 1, kEpiSwiglu = 2, kEpiResidual = 3;
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// y carries no __restrict__: in residual mode `resid` may be y itself.
 template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
 __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
-                     const uint16_t *__restrict__ scales, float *__restrict__ y, int m, int n,
+                     const uint16_t *__restrict__ scales, float *y, int m, int n,
                      int k, int stages, int stage_bytes, int x_bytes,
                      unsigned long long *__restrict__ keys = nullptr, const float *resid = nullptr) {
   constexpr int kBulkWarps = NW;
