@@ -1,27 +1,29 @@
 """Benchmark of the weight-only block-32 qgemv/qgemm path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-Default workload ("decoder_block_m1"): one Qwen3-0.6B-style decoder block at decode, M = 1,
+Headline workload ("decoder_block_m1"): one Qwen3-0.6B-style decoder block at decode, M = 1,
 int4 block-32 weights: the 7 projections q[2048x1024], k[1024x1024], v[1024x1024],
 o[1024x2048], gate/up[3072x1024], down[1024x3072]. q|k|v share their input, as do gate|up,
 so their packed rows are stored concatenated and one step is 4 qgemv calls: qkv[4096x1024],
 o, gate_up[6144x1024], down (--unfused: 7 calls). Consecutive steps walk the 28 blocks of a
-seeded synthetic decoder (247.7 MB of packed weights, more than the 126 MB L2), so every
-step streams its weights from HBM. Metric: weight GB/s (packed codes + scales per step /
-time).
+seeded synthetic decoder (247.7 MB of packed weights, more than the 126 MB L2), and L2 is
+flushed before the timed region, so every step streams its weights from HBM. Metric: weight
+GB/s (packed codes + scales per step / time).
 
 Timed region: K steps replayed from CUDA graphs on one stream, bracketed by a barrier and
-device synchronisation, timed with CUDA events on that stream; the max over ranks is
-reported. Under torchrun every rank runs its own replica (no data-path collective).
+device synchronisation, timed with CUDA events on that stream; every graph the timed region
+replays has been replayed once, untimed, before it; the max over ranks is reported. Under
+torchrun every rank runs its own replica (no data-path collective).
 
-Also on the JSON line: `e2e` (the same steps through the public API with x copied from
-pinned host memory and y read back every step), `roofline` (the qgemv kernel against the
-measured HBM copy bandwidth), `cpu_baseline` (the CPU oracle on the host cores, a bounded
-sample), `parity` (GPU vs oracle on the sampled step), `kernel_roofline_lm_head` (one qgemv
-launch over the 165 MB int8 lm_head, the kernel alone against HBM), and `prefill` (the tcgen05
-qgemm over all projections of all 28 blocks at M = 512, TFLOP/s against the measured bf16
-peak).
+Also on the JSON line: `per_kernel` (each projection's launch timed alone, L2-cold), `e2e`
+(the same steps through the public API with x copied from pinned host memory and y read back
+every step), `roofline` (the decode kernel against the measured HBM copy bandwidth),
+`cpu_baseline` (the CPU oracle on the host cores, all cores and one core, a bounded sample),
+`parity` (GPU vs oracle on the sampled step), and `configs`: one object per workload
+configuration of the benchmark (a single qgemv; the decoder block; the int8 lm_head; prefill
+M = 512 over all 28 blocks; batched decode M = 64 and prefill M = 4096 over all 28 blocks
+plus the lm_head), each with its own dtype, roofline and CPU baseline.
 """
 
 from __future__ import annotations
@@ -45,6 +47,7 @@ from weight_only_bit_qgemv_b200 import workloads  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
+METRIC = "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)"
 
 
 def measured_traffic(workload: str, root: str | None = None):
@@ -193,6 +196,107 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------------------
+# timing helpers
+# --------------------------------------------------------------------------------------
+
+class L2Flush:
+    """Writes a buffer twice the size of L2, so that what follows starts with L2 cold."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    def __call__(self, stream):
+        with torch.cuda.stream(stream):
+            self.buf.fill_(1.0)
+
+
+def capture_graph(fn, count, stream, start=0):
+    """CUDA graph of fn(start), ..., fn(start + count - 1); returns (graph, our launches)."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    g = torch.cuda.CUDAGraph()
+    c0 = woq.launch_count()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(count):
+            fn(start + i)
+    return g, woq.launch_count() - c0
+
+
+def time_replays(graphs, stream, world, flush):
+    """Device ms of replaying `graphs` in order, timed with CUDA events on `stream`.
+
+    Every distinct graph is replayed once, untimed, first (its upload and first-launch costs
+    stay out of the timed region); then L2 is flushed, the ranks meet at a barrier, and the
+    replays run between two events, with a device synchronisation on both sides."""
+    seen = []
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            if all(g is not h for h in seen):
+                g.replay()
+                seen.append(g)
+    flush(stream)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for g in graphs:
+            g.replay()
+        end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end)
+
+
+def time_graph_steps(step_fn, n_cycle: int, steps: int, warmup: int, stream, world, flush):
+    """Time `steps` steps of step_fn(i % n_cycle), replayed from CUDA graphs.
+
+    Graphs: `full` holds steps 0..n_cycle-1, `rem` steps 0..(steps % n_cycle)-1; the timed
+    region replays full (steps // n_cycle) times, then rem. Untimed first: each of them once,
+    and full again until at least `warmup` steps have run. Returns (ms, our launches per step).
+    """
+    with torch.cuda.stream(stream):
+        for i in range(min(2, n_cycle)):  # eager warm-up (attribute setup, lazy module loads)
+            step_fn(i)
+    stream.synchronize()
+    full, launches_full = capture_graph(step_fn, n_cycle, stream)
+    rem = steps % n_cycle
+    g_rem = capture_graph(step_fn, rem, stream)[0] if rem else None
+    timed = [full] * (steps // n_cycle) + ([g_rem] if g_rem is not None else [])
+    done = (n_cycle if steps >= n_cycle else 0) + rem
+    with torch.cuda.stream(stream):
+        while done < warmup:
+            full.replay()
+            done += n_cycle
+    ms = time_replays(timed, stream, world, flush)
+    del full, g_rem
+    return ms, launches_full / n_cycle
+
+
+def time_graph_median(fn, count, stream, world, flush, reps=3):
+    """Median over `reps` of the device ms of one replay of a graph of fn(0..count-1), each
+    replay after an L2 flush. Returns (median ms, our launches per replay)."""
+    with torch.cuda.stream(stream):
+        fn(0)
+    stream.synchronize()
+    g, launches = capture_graph(fn, count, stream)
+    times = [time_replays([g], stream, world, flush) for _ in range(reps)]
+    del g
+    return statistics.median(times), launches
+
+
+def roofline(achieved, peak, unit, bound, peak_kind, traffic=None, **extra):
+    out = {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+           "frac": round(achieved / peak, 4), "traffic": traffic,
+           "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else peak_kind}
+    out.update(extra)
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # the workload
 # --------------------------------------------------------------------------------------
 
@@ -234,58 +338,12 @@ def decode_step_bytes(layer):
     return sum(w.nbytes for w in layer)
 
 
-def time_graph_steps(step_fn, n_cycle: int, steps: int, warmup: int, stream, world):
-    """Capture step_fn(i) for i in [0, n_cycle) into a graph; replay to cover `steps` steps.
-
-    Returns (ms for the K timed steps, launches of our kernels per step).
-    """
-    import weight_only_bit_qgemv_b200 as woq
-
-    def capture(count, start):
-        g = torch.cuda.CUDAGraph()
-        c0 = woq.launch_count()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(count):
-                step_fn((start + i) % n_cycle)
-        return g, woq.launch_count() - c0
-
-    with torch.cuda.stream(stream):
-        for i in range(min(2, n_cycle)):  # eager warm-up (allocations, attribute setup)
-            step_fn(i)
-    stream.synchronize()
-    full, launches_full = capture(n_cycle, 0)
-    rem = steps % n_cycle
-    g_rem = capture(rem, 0)[0] if rem else None
-    per_step = launches_full / n_cycle
-
-    # warm-up steps, untimed
-    w_full, w_rem = divmod(warmup, n_cycle)
-    g_wrem = capture(w_rem, 0)[0] if w_rem else None
-    with torch.cuda.stream(stream):
-        for _ in range(w_full):
-            full.replay()
-        if g_wrem is not None:
-            g_wrem.replay()
-    stream.synchronize()
-
-    barrier(world)
-    torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(steps // n_cycle):
-            full.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        end.record(stream)
-    end.synchronize()
-    torch.cuda.synchronize()
-    barrier(world)
-    return start.elapsed_time(end), per_step
+def block_flops(m):
+    return 2.0 * m * sum(n * k for _, n, k in workloads.DECODER_PROJ)
 
 
-def run_decode(args, world, rank, local, peaks, peak_kind):
+def run_decode(args, world, local, peaks, peak_kind, flush):
+    """Configuration 2 (the headline): one decoder block per step at M = args.m."""
     import weight_only_bit_qgemv_b200 as woq
 
     device = torch.device("cuda", local)
@@ -305,26 +363,45 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
 
     stream = torch.cuda.Stream(device)
     with ClockSampler(local) as clk:
-        ms, per_step = time_graph_steps(step, len(layers), args.steps, args.warmup, stream, world)
+        ms, per_step = time_graph_steps(step, len(layers), args.steps, args.warmup, stream, world,
+                                        flush)
     clocks = clk.summary()
     value, ms_max = aggregate_throughput(step_bytes * args.steps, ms, world)
     gbs = value / 1e9
 
-    # the qgemv kernel against the HBM roofline: every launch in the timed region is it
+    # Each projection's launch alone: a graph of it over the 28 blocks, after an L2 flush.
+    per_kernel = []
+    for g, (nm, mem) in enumerate(groups):
+        def one(i, g=g):
+            woq.qgemv(xs[g], layers[i % len(layers)][g], out=ys[g])
+
+        kms, _ = time_graph_median(one, len(layers), stream, world, flush)
+        us = kms * 1e3 / len(layers)
+        nb = layers[0][g].nbytes
+        per_kernel.append({"launch": f"{nm}[{group_shape(mem)[0]}x{group_shape(mem)[1]}]",
+                           "us": round(us, 3), "weight_bytes": nb,
+                           "gbs": round(nb / (us * 1e-6) / 1e9, 1),
+                           "hbm_frac": round(nb / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)})
+    sum_us = sum(p["us"] for p in per_kernel)
+    step_us = ms * 1e3 / args.steps
+    dom = max(per_kernel, key=lambda p: p["us"])
+
+    # The decode kernel against the HBM roofline: every launch in the timed region is a
+    # qgemv launch; achieved = algorithmic bytes per launch / the timed region's average launch.
     launches = per_step * args.steps
     achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": (measured_traffic("decoder_block_m1")
-                            if M == 1 and not args.unfused else None),
-                "peak_source": peak_kind,
-                "bytes_per_launch": round(step_bytes / per_step),
-                "avg_launch_us": round(ms * 1e3 / launches, 3)}
+    roof = roofline(achieved, peaks["hbm_gbs"], "GB/s", "hbm", peak_kind,
+                    traffic=(measured_traffic("decoder_block_m1") if M == 1 and not args.unfused
+                             else None),
+                    bytes_per_launch=round(step_bytes / per_step),
+                    avg_launch_us=round(ms * 1e3 / launches, 3),
+                    dominant_kernel={"launch": dom["launch"], "us_alone": dom["us"],
+                                     "gbs_alone": dom["gbs"], "frac_alone": dom["hbm_frac"]})
 
     e2e = run_decode_e2e(layers, groups, device, min(args.steps, 2000), stream, world, M)
 
     out = {
-        "metric": "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)",
+        "metric": METRIC,
         "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -333,7 +410,7 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
                                 for nm, mem in groups],
                    "fused_qkv_gate_up": not args.unfused,
                    "layers_cycled": len(layers), "weight_bytes_per_step": step_bytes,
-                   "l2": f"inputs larger than L2: steps walk {len(layers)} blocks, "
+                   "l2": f"L2 flushed before the timed region, and steps walk {len(layers)} blocks, "
                          f"{total_bytes / 1e6:.1f} MB of packed weights > 126 MB L2",
                    "launch": "CUDA graph of qgemv C-ABI calls, programmatic dependent launch",
                    "parallelism": f"replicas x{world}"},
@@ -341,7 +418,12 @@ def run_decode(args, world, rank, local, peaks, peak_kind):
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": int(launches),
-        "roofline": roofline,
+        "roofline": roof,
+        "per_kernel": {"timing": "each launch group alone: a CUDA graph of its 28 blocks' launches "
+                                 "after an L2 flush, median of 3, per launch",
+                       "kernels": per_kernel, "sum_us": round(sum_us, 3),
+                       "step_us": round(step_us, 3),
+                       "share_of_step": {p["launch"]: round(p["us"] / step_us, 3) for p in per_kernel}},
     }
     return out, layers, groups, xs
 
@@ -390,7 +472,7 @@ def run_decode_e2e(layers, groups, device, steps, stream, world, M=1):
             graphs[i % len(graphs)].replay()
             stream.synchronize()
 
-        for i in range(5):
+        for i in range(len(graphs)):  # every graph replayed once, untimed
             step(i)
         barrier(world)
         torch.cuda.synchronize()
@@ -411,16 +493,56 @@ def run_decode_e2e(layers, groups, device, steps, stream, world, M=1):
                       "one pinned-memory copy each way; the host waits for each step's outputs"}
 
 
-def run_lm_head_roofline(device, peaks, peak_kind, reps=20):
-    """qgemv on the int8 lm_head [151936x1024] at M = 1: one 165 MB launch, the kernel alone.
+def run_single_qgemv(device, peaks, peak_kind, stream, world, flush):
+    """Configuration 1: one qgemv, x [1, 1024], W [3072, 1024] int4 (W seed 0, x seed 0).
 
-    Two packed copies alternate so that every launch streams its weights from HBM.
-    """
+    The weight is 1.77 MB, far below L2, so a CUDA graph of calls rotates over distinct copies
+    of it whose total is more than twice L2: every call streams its weights from HBM. Reported:
+    the average call in that graph (programmatic dependent launch between calls), and the
+    latency of one call alone (L2 flushed first, the GPU kept busy while it is enqueued)."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    n, k = 3072, 1024
+    w0 = woq.pack(workloads.weight(n, k, seed=0), 4, device)
+    copies = -(-2 * L2_BYTES // w0.nbytes) + 1
+    ws = [w0] + [woq.PackedWeight(w0.packed.clone(), w0.scales.clone(), 4, n, k)
+                 for _ in range(copies - 1)]
+    x = workloads.activations(1, k, seed=0).to(device)
+    y = torch.empty(1, n, device=device)
+    ms, launches = time_graph_median(lambda i: woq.qgemv(x, ws[i % copies], out=y), copies,
+                                     stream, world, flush)
+    call_us = ms * 1e3 / copies
+    # one call alone
+    lat = []
+    with torch.cuda.stream(stream):
+        for r in range(7):
+            flush(stream)
+            torch.cuda._sleep(40000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            woq.qgemv(x, ws[r % copies], out=y, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            lat.append(e0.elapsed_time(e1) * 1e3)
+    gbs = w0.nbytes / (call_us * 1e-6) / 1e9
+    return {"workload": "single_qgemv_m1_int4_3072x1024", "dtype": "f32", "weight_bytes": w0.nbytes,
+            "us_per_call": round(call_us, 3), "gbs": round(gbs, 1),
+            "single_call_latency_us": round(statistics.median(lat), 3),
+            "calls_in_graph": copies, "launches_per_call": launches / copies,
+            "timing": f"CUDA graph of {copies} calls rotating over {copies} copies "
+                      f"({copies * w0.nbytes / 1e6:.0f} MB > 2x L2), after an L2 flush, median of 3; "
+                      "single call: median of 7, each after an L2 flush",
+            "roofline": roofline(gbs, peaks["hbm_gbs"], "GB/s", "hbm", peak_kind)}
+
+
+def run_lm_head(device, peaks, peak_kind, bits, reps=20):
+    """Configuration 3: qgemv on the lm_head [151936x1024] at M = 1: one 165 MB (int8) launch,
+    the kernel alone; two packed copies alternate so that every launch streams from HBM."""
     import weight_only_bit_qgemv_b200 as woq
 
     n, k = workloads.LM_HEAD
-    w0 = woq.pack(workloads.weight(n, k, seed=workloads.LM_HEAD_SEED), 8, device)
-    w1 = woq.PackedWeight(w0.packed.clone(), w0.scales.clone(), 8, n, k)
+    w0 = woq.pack(workloads.weight(n, k, seed=workloads.LM_HEAD_SEED), bits, device)
+    w1 = woq.PackedWeight(w0.packed.clone(), w0.scales.clone(), bits, n, k)
     x = workloads.activations(1, k, seed=workloads.X_SEED).to(device)
     y = torch.empty(1, n, device=device)
     for _ in range(3):
@@ -437,104 +559,141 @@ def run_lm_head_roofline(device, peaks, peak_kind, reps=20):
     times = [ev[r].elapsed_time(ev[r + 1]) for r in range(reps)]
     med = statistics.median(times)
     gbs = w0.nbytes / (med / 1e3) / 1e9
-    # The fused greedy pick over the same weights (zero keys, GEMV with argmax, finish):
-    # no logits written.
-    # Timed as a decode loop runs it: calls captured in a CUDA graph (programmatic dependent
-    # launch between the three kernels), replayed.
-    gs = torch.cuda.Stream(device)
-    for _ in range(3):
-        woq.qgemv_argmax(x, w0, stream=gs)
-    gs.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=gs):
-        for r in range(reps):
-            woq.qgemv_argmax(x, w0 if r % 2 == 0 else w1, stream=gs)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(gs):  # replay() launches on the current stream
-        for _ in range(2):
-            graph.replay()
+    out = {"workload": f"lm_head_m1_int{bits}", "dtype": "f32", "weight_bytes": w0.nbytes,
+           "launch_us_median": round(med * 1e3, 3), "gbs": round(gbs, 1),
+           "timing": f"median of {reps} single launches, CUDA events, two alternating copies",
+           "roofline": roofline(gbs, peaks["hbm_gbs"], "GB/s", "hbm", peak_kind,
+                                traffic=measured_traffic(f"lm_head_m1_int{bits}"))}
+    if bits == 8:
+        # The fused greedy pick over the same weights (zero keys, GEMV with argmax, finish):
+        # no logits written. Timed as a decode loop runs it: calls captured in a CUDA graph
+        # (programmatic dependent launch between the three kernels), replayed.
+        gs = torch.cuda.Stream(device)
+        for _ in range(3):
+            woq.qgemv_argmax(x, w0, stream=gs)
         gs.synchronize()
-        e0.record(gs)
-        graph.replay()
-        e1.record(gs)
-    e1.synchronize()
-    amed = e0.elapsed_time(e1) / reps
-    del graph
-    argmax = {"call_us": round(amed * 1e3, 2), "achieved": round(w0.nbytes / (amed / 1e3) / 1e9, 1),
-              "unit": "GB/s", "launches_per_call": 3,
-              "timing": f"{reps} calls replayed from one CUDA graph, CUDA events"}
-    return {"workload": "lm_head_m1_int8", "weight_bytes": w0.nbytes, "launch_us_median": med * 1e3,
-            "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "traffic": measured_traffic("lm_head_m1_int8"),
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peak_kind,
-            "timing": f"median of {reps} single launches, CUDA events, two alternating copies",
-            "greedy_argmax": argmax}
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            for r in range(reps):
+                woq.qgemv_argmax(x, w0 if r % 2 == 0 else w1, stream=gs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(gs):  # replay() launches on the current stream
+            for _ in range(2):
+                graph.replay()
+            gs.synchronize()
+            e0.record(gs)
+            graph.replay()
+            e1.record(gs)
+        e1.synchronize()
+        amed = e0.elapsed_time(e1) / reps
+        del graph
+        out["greedy_argmax"] = {"call_us": round(amed * 1e3, 2),
+                                "gbs": round(w0.nbytes / (amed / 1e3) / 1e9, 1),
+                                "launches_per_call": 3,
+                                "timing": f"{reps} calls replayed from one CUDA graph, CUDA events"}
+    return out
 
 
-def run_prefill(layers, groups, device, m: int, reps: int, peaks, peak_kind, world):
-    """tcgen05 qgemm through every projection of every block at M = m (one pass = one rep)."""
+def run_prefill(layers, groups, device, m: int, peaks, peak_kind, stream, world, flush,
+                lm_head=None):
+    """tcgen05 qgemm through every projection of every block at M = m (one pass), plus the
+    int8 lm_head if given. Median of 3 passes, each replayed from a CUDA graph after an L2
+    flush."""
     import weight_only_bit_qgemv_b200 as woq
 
     Xs = [workloads.activations(m, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
           for _, mem in groups]
     Ys = [torch.empty(m, group_shape(mem)[0], device=device) for _, mem in groups]
-    ws = torch.empty(max(woq.qgemm_workspace_bytes(m, w, "bf16_tc") for w in layers[0]),
-                     dtype=torch.uint8, device=device)
-    flops = 2.0 * m * sum(n * k for _, n, k in workloads.DECODER_PROJ) * len(layers)
+    ws_need = [woq.qgemm_workspace_bytes(m, w, "bf16_tc") for w in layers[0]]
+    flops = block_flops(m) * len(layers)
+    if lm_head is not None:
+        X_lm = workloads.activations(m, lm_head.k, seed=workloads.X_SEED).to(device)
+        Y_lm = torch.empty(m, lm_head.n, device=device)
+        ws_need.append(woq.qgemm_workspace_bytes(m, lm_head, "bf16_tc"))
+        flops += 2.0 * m * lm_head.n * lm_head.k
+    ws = torch.empty(max(ws_need), dtype=torch.uint8, device=device)
 
-    def step(i):
+    def pass_(i):
         for layer in layers:
             for g, w in enumerate(layer):
                 woq.qgemm(Xs[g], w, path="bf16_tc", out=Ys[g], workspace=ws)
+        if lm_head is not None:
+            woq.qgemm(X_lm, lm_head, path="bf16_tc", out=Y_lm, workspace=ws)
 
-    stream = torch.cuda.Stream(device)
-    ms, per_step = time_graph_steps(step, 1, reps, 2, stream, world)
-    tflops = flops * reps / (ms / 1e3) / 1e12
-    return {"workload": f"prefill_m{m}", "m": m, "gemm_calls_per_pass": len(layers) * len(groups),
-            "flop_per_pass": flops, "passes": reps, "ms_per_pass": ms / reps,
-            "tflops": round(tflops, 1), "peak_tflops": peaks["bf16_tflops"],
-            "frac": round(tflops / peaks["bf16_tflops"], 4), "peak_source": peak_kind,
-            "launches_per_pass": int(per_step)}
+    ms, launches = time_graph_median(pass_, 1, stream, world, flush)
+    tflops = flops / (ms / 1e3) / 1e12
+    calls = len(layers) * len(groups) + (1 if lm_head is not None else 0)
+    return {"workload": f"prefill_m{m}" + ("_plus_lm_head" if lm_head is not None else ""),
+            "dtype": "bf16 operands, f32 accumulate", "m": m, "gemm_calls_per_pass": calls,
+            "flop_per_pass": flops, "ms_per_pass": round(ms, 4), "tflops": round(tflops, 1),
+            "launches_per_pass": int(launches),
+            "timing": "one pass replayed from a CUDA graph after an L2 flush, median of 3",
+            "roofline": roofline(tflops, peaks["bf16_tflops"], "TFLOP/s", "tensor", peak_kind,
+                                 peak_note="bf16 burst (kernel timed alone)")}
 
 
-def run_batched_decode(layers, groups, device, m: int, steps: int, peaks, peak_kind, world):
+def run_batched_decode(layers, groups, device, m: int, peaks, peak_kind, stream, world, flush,
+                       lm_head=None):
     """Batched decode: m activation rows through every fused projection of every block via
-    qgemm's automatic path (the FP32-accurate split tensor-core GEMM for 24 <= m < 128, the
-    CUDA-core kernel below), replayed from CUDA graphs like the M = 1 decode."""
+    qgemm's automatic path (the FP32-accurate split tensor-core GEMM for 24 <= m < 128), then
+    the int8 lm_head if given. One decoder step = 28 blocks (+ lm_head), replayed from a CUDA
+    graph after an L2 flush, median of 3."""
     import weight_only_bit_qgemv_b200 as woq
 
     xs = [workloads.activations(m, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
           for _, mem in groups]
     ys = [torch.empty(m, group_shape(mem)[0], device=device) for _, mem in groups]
-    need = max(woq.qgemm_workspace_bytes(m, w, "auto") for w in layers[0])
-    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    need = [woq.qgemm_workspace_bytes(m, w, "auto") for w in layers[0]]
+    if lm_head is not None:
+        x_lm = workloads.activations(m, lm_head.k, seed=workloads.X_SEED).to(device)
+        y_lm = torch.empty(m, lm_head.n, device=device)
+        need.append(woq.qgemm_workspace_bytes(m, lm_head, "auto"))
+    ws = torch.empty(max(max(need), 256), dtype=torch.uint8, device=device)
 
-    def step(i):
-        for g, w in enumerate(layers[i]):
+    def blocks_only(i):
+        for g, w in enumerate(layers[i % len(layers)]):
             woq.qgemm(xs[g], w, path="auto", out=ys[g], workspace=ws)
 
-    stream = torch.cuda.Stream(device)
-    ms, per_step = time_graph_steps(step, len(layers), steps, max(3, steps // 10), stream, world)
-    us_block = ms * 1e3 / steps
+    ms_blocks, launches_blocks = time_graph_median(blocks_only, len(layers), stream, world, flush)
+    us_block = ms_blocks * 1e3 / len(layers)
     step_bytes = decode_step_bytes(layers[0])
-    flops = 2.0 * m * sum(n * k for _, n, k in workloads.DECODER_PROJ)
+    block_gbs = step_bytes / (us_block * 1e-6) / 1e9
     path = "split_tc" if 24 <= m < 128 else ("bf16_tc" if m >= 128 else "fp32")
-    return {"workload": f"decoder_block_m{m}", "m": m, "qgemm_path": path,
-            "blocks_timed": steps, "us_per_block": round(us_block, 2),
-            "tokens_per_s": round(m * 1e6 / (us_block * len(layers)), 1),
-            "weight_gbs": round(step_bytes / (us_block * 1e-6) / 1e9, 1),
-            "hbm_frac": round(step_bytes / (us_block * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
-            "algorithmic_tflops": round(flops / (us_block * 1e-6) / 1e12, 2),
-            "peak_source": peak_kind, "launches_per_block": int(per_step)}
+    out = {"workload": f"decoder_m{m}" + ("_plus_lm_head" if lm_head is not None else ""),
+           "dtype": "f32 (split tensor-core form: bf16 hi+lo operands, f32 accumulate)"
+                    if path == "split_tc" else "f32",
+           "m": m, "qgemm_path": path, "us_per_block": round(us_block, 2),
+           "launches_per_block": launches_blocks / len(layers),
+           "block_weight_gbs": round(block_gbs, 1),
+           "block_algorithmic_tflops": round(block_flops(m) / (us_block * 1e-6) / 1e12, 2)}
+    total_bytes = step_bytes * len(layers)
+    total_us = us_block * len(layers)
+    if lm_head is not None:
+        def lm(i):
+            woq.qgemm(x_lm, lm_head, path="auto", out=y_lm, workspace=ws)
+
+        ms_lm, _ = time_graph_median(lm, 1, stream, world, flush)
+        out["lm_head_us"] = round(ms_lm * 1e3, 2)
+        out["lm_head_gbs"] = round(lm_head.nbytes / (ms_lm * 1e-3) / 1e9, 1)
+        total_bytes += lm_head.nbytes
+        total_us += ms_lm * 1e3
+    gbs = total_bytes / (total_us * 1e-6) / 1e9
+    out.update({"decoder_step_us": round(total_us, 1),
+                "tokens_per_s": round(m * 1e6 / total_us, 1),
+                "weight_gbs": round(gbs, 1),
+                "timing": "blocks: a CUDA graph of the 28 blocks' calls after an L2 flush, median "
+                          "of 3; lm_head: one call, same rule",
+                "roofline": roofline(gbs, peaks["hbm_gbs"], "GB/s", "hbm", peak_kind)})
+    return out
 
 
-def run_fused_epilogues(layers, groups, device, steps: int, world):
-    """The decode-step projections whose neighbours fuse (NEXT-4 rows): gate|up with the SwiGLU
+def run_fused_epilogues(layers, groups, device, stream, world, flush):
+    """The decode-step projections whose neighbours fuse: gate|up with the SwiGLU
     (qgemv_swiglu, the gate|up outputs never written) and down with the residual add
     (qgemv_residual, in place on the hidden state), each against the plain qgemv of the same
-    weights; M = 1, all 28 blocks cycled, CUDA graphs as the decode steps. Timing only: the
-    decode step's gate|up matrix is packed as gate rows then up rows, not interleaved, which
-    changes which rows pair up but not the work."""
+    weights; M = 1, all 28 blocks cycled. Timing only: the decode step's gate|up matrix is
+    packed as gate rows then up rows, not interleaved, which changes which rows pair up but
+    not the work."""
     import weight_only_bit_qgemv_b200 as woq
 
     names = [nm for nm, _ in groups]
@@ -549,19 +708,18 @@ def run_fused_epilogues(layers, groups, device, steps: int, world):
     y_sw = torch.empty(1, n_gu // 2, device=device)
     h = torch.zeros(1, n_dn, device=device)
     y_dn = torch.empty(1, n_dn, device=device)
-    stream = torch.cuda.Stream(device)
-    warm = max(3, steps // 10)
+    nl = len(layers)
 
     def timed(fn):
-        ms, per_step = time_graph_steps(fn, len(layers), steps, warm, stream, world)
-        return ms * 1e3 / steps, int(per_step)
+        ms, launches = time_graph_median(fn, nl, stream, world, flush)
+        return ms * 1e3 / nl, launches / nl
 
-    out = {"m": 1, "calls_timed": steps}
+    out = {"m": 1}
     for key, plain, fused, idx in (
-        ("swiglu_gate_up", lambda i: woq.qgemv(x_gu, layers[i][gu], out=y_gu),
-         lambda i: woq.qgemv_swiglu(x_gu, layers[i][gu], out=y_sw), gu),
-        ("residual_down", lambda i: woq.qgemv(x_dn, layers[i][dn], out=y_dn),
-         lambda i: woq.qgemv_residual(x_dn, layers[i][dn], h, out=h), dn),
+        ("swiglu_gate_up", lambda i: woq.qgemv(x_gu, layers[i % nl][gu], out=y_gu),
+         lambda i: woq.qgemv_swiglu(x_gu, layers[i % nl][gu], out=y_sw), gu),
+        ("residual_down", lambda i: woq.qgemv(x_dn, layers[i % nl][dn], out=y_dn),
+         lambda i: woq.qgemv_residual(x_dn, layers[i % nl][dn], h, out=h), dn),
     ):
         nbytes = layers[0][idx].nbytes
         us_plain, _ = timed(plain)
@@ -573,7 +731,7 @@ def run_fused_epilogues(layers, groups, device, steps: int, world):
 
 
 # --------------------------------------------------------------------------------------
-# CPU oracle (cpu_baseline leg and the reference arm)
+# CPU oracle (cpu_baseline legs and the reference arm)
 # --------------------------------------------------------------------------------------
 
 def oracle_decode_pass(packed_layer, xs_np, rows=None):
@@ -588,22 +746,34 @@ def oracle_decode_pass(packed_layer, xs_np, rows=None):
     return outs
 
 
-def oracle_layer_inputs(groups, bits=4, layer=0):
-    """The block's 7 projections, quantised and packed by the oracle itself, and their x rows
-    (members of a launch group share its input)."""
+def oracle_pack(W: np.ndarray, bits: int):
+    """(packed, scale bits, bits) of a float32 weight, quantised and packed by the oracle."""
     import oracle
 
+    q, s = oracle.quantise(W, bits)
+    return oracle.pack(q, bits), s, bits
+
+
+def oracle_layer_inputs(groups, bits=4, layer=0, m=1):
+    """The block's 7 projections, quantised and packed by the oracle itself, and their x rows
+    (members of a launch group share its input)."""
     x_of = {}
     for _, mem in groups:
-        x = workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).numpy()
+        x = workloads.activations(m, group_shape(mem)[1], seed=group_x_seed(mem)).numpy()
         for i in mem:
             x_of[i] = x
     out = []
     for p, (_, n, k) in enumerate(workloads.DECODER_PROJ):
         W = workloads.weight(n, k, seed=workloads.layer_seed(layer, p)).numpy()
-        q, s = oracle.quantise(W, bits)
-        out.append((oracle.pack(q, bits), s, bits))
+        out.append(oracle_pack(W, bits))
     return out, [x_of[p] for p in range(len(workloads.DECODER_PROJ))]
+
+
+def all_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def blas_threads():
@@ -616,37 +786,92 @@ def blas_threads():
         return 1
 
 
-def time_oracle(packed_layer, xs, budget_s: float):
-    """Median seconds per decode-block pass of the oracle; the outputs of the last pass."""
-    oracle_decode_pass(packed_layer, xs)  # discarded warm-up
-    times, outs = [], None
-    t_end = time.perf_counter() + budget_s
-    while len(times) < 3 or time.perf_counter() < t_end:
-        t0 = time.perf_counter()
-        outs = oracle_decode_pass(packed_layer, xs)
-        times.append(time.perf_counter() - t0)
-        if len(times) >= 50:
-            break
-    return statistics.median(times), len(times), outs
+def time_cpu(fn, threads: int, runs: int = 3):
+    """Median seconds of fn() with BLAS limited to `threads` threads: one discarded run, then
+    the median of `runs`. Returns (seconds, threads actually used, last result)."""
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=threads, user_api="blas"):
+        used = blas_threads()
+        res = fn()
+        ts = []
+        for _ in range(runs):
+            t0 = time.perf_counter()
+            res = fn()
+            ts.append(time.perf_counter() - t0)
+    return statistics.median(ts), used, res
 
 
-def cpu_baseline_leg(layer0_gpu, groups, xs_gpu, budget_s):
+def cpu_baseline(fn, work: float, unit: str, scale: float, sample: str):
+    """The oracle timed on all host cores and on one core. `work` units per run (bytes or
+    FLOP), reported in `unit` after dividing by `scale` (1e9 for GB/s, 1e12 for TFLOP/s)."""
+    n_all = all_cores()
+    sec_all, used_all, res = time_cpu(fn, n_all)
+    sec_one, used_one, _ = time_cpu(fn, 1)
+    return ({"value": round(work / sec_all / scale, 5), "unit": unit, "cores": used_all,
+             "kind": "oracle", "sample": sample,
+             "seconds_per_run": round(sec_all, 4),
+             "one_core": {"value": round(work / sec_one / scale, 5), "cores": used_one,
+                          "seconds_per_run": round(sec_one, 4)},
+             "timing": "one discarded run, then the median of 3 (all cores in the affinity set, "
+                       "then BLAS limited to one thread)"}, res)
+
+
+def cpu_legs(groups, layer0_gpu, xs_gpu):
+    """The oracle as it stands on the host cores, one bounded sample per configuration; also the
+    parity of the headline GPU step against the oracle's outputs (block 0)."""
+    import oracle
     import weight_only_bit_qgemv_b200 as woq
 
+    legs = {}
+    # configuration 1: the single qgemv, in full
+    n, k = 3072, 1024
+    pk1 = oracle_pack(workloads.weight(n, k, seed=0).numpy(), 4)
+    x1 = workloads.activations(1, k, seed=0).numpy()
+    b1 = pk1[0].nbytes + pk1[1].nbytes
+    legs["single_qgemv_m1"], _ = cpu_baseline(
+        lambda: oracle.qgemv_ref(x1, *pk1), b1, "GB/s", 1e9,
+        "the whole [3072x1024] int4 qgemv at M=1 through the NumPy float64 oracle")
+    # configuration 2: decoder block 0, in full (and parity of the GPU step)
     packed, xs = oracle_layer_inputs(groups)
-    sec, passes, outs = time_oracle(packed, xs, budget_s)
     nbytes = sum(pk.nbytes + sc.nbytes for pk, sc, _ in packed)
-    # parity of the GPU step against the oracle on the same inputs (block 0)
+    legs["decoder_block_m1"], outs = cpu_baseline(
+        lambda: oracle_decode_pass(packed, xs), nbytes, "GB/s", 1e9,
+        "decoder block 0 (7 projections, M=1, int4) through the NumPy float64 oracle")
     errs = []
     for g, (w, (_, mem)) in enumerate(zip(layer0_gpu, groups)):
         y = woq.qgemv(xs_gpu[g], w).cpu().numpy()
         ref = np.concatenate([outs[i] for i in mem], axis=1)
         errs.append(float(np.max(np.abs(y - ref)) / np.max(np.abs(ref))))
-    return ({"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
-             "kind": "oracle",
-             "sample": f"{passes} passes of decoder block 0 (7 projections, M=1, int4) through the "
-                       f"NumPy float64 oracle, median pass {sec * 1e3:.1f} ms"},
-            {"max_rel_err": max(errs), "tolerance": 1e-4, "checked": "block 0, every output"})
+    parity = {"max_rel_err": max(errs), "tolerance": 1e-4, "checked": "block 0, every output"}
+    # configuration 3: lm_head int8, the first 8192 of its 151936 rows
+    rows = 8192
+    n, k = workloads.LM_HEAD
+    W = workloads.weight(n, k, seed=workloads.LM_HEAD_SEED)[:rows].numpy()
+    pk3 = oracle_pack(W, 8)
+    x3 = workloads.activations(1, k, seed=workloads.X_SEED).numpy()
+    legs["lm_head_m1_int8"], _ = cpu_baseline(
+        lambda: oracle.qgemv_ref(x3, *pk3), pk3[0].nbytes + pk3[1].nbytes, "GB/s", 1e9,
+        f"rows 0..{rows - 1} of the int8 lm_head [151936x1024] at M=1 (the rate is per byte, "
+        "so it stands for the whole matrix)")
+    # configuration 4: prefill M=512, block 0's 7 projections (1/28 of a pass)
+    packed512, xs512 = oracle_layer_inputs(groups, m=512)
+    legs["prefill_m512"], _ = cpu_baseline(
+        lambda: oracle_decode_pass(packed512, xs512), block_flops(512), "TFLOP/s", 1e12,
+        "decoder block 0's 7 projections at M=512 (1/28 of the pass; a rate, so it stands for "
+        "the pass)")
+    # configuration 5: batched decode M=64 (block 0) and prefill M=4096 (block 0's q projection)
+    packed64, xs64 = oracle_layer_inputs(groups, m=64)
+    legs["decoder_m64"], _ = cpu_baseline(
+        lambda: oracle_decode_pass(packed64, xs64), nbytes, "GB/s", 1e9,
+        "decoder block 0's 7 projections at M=64 (weight bytes per second; a rate, so it stands "
+        "for the 28 blocks)")
+    q0 = packed[0]
+    x4096 = workloads.activations(4096, 1024, seed=workloads.X_SEED).numpy()
+    legs["prefill_m4096"], _ = cpu_baseline(
+        lambda: oracle.qgemv_ref(x4096, *q0), 2.0 * 4096 * 2048 * 1024, "TFLOP/s", 1e12,
+        "block 0's q projection [2048x1024] at M=4096 (a rate, so it stands for the pass)")
+    return legs, parity
 
 
 def run_reference(args, world, rank, budget_s=90.0):
@@ -675,8 +900,7 @@ def run_reference(args, world, rank, budget_s=90.0):
     sample = (f"each step: rows {rows} of the 7 projections of decoder block 0 (M=1, int4), "
               f"{nbytes} weight bytes, through the NumPy float64 oracle; one full block pass "
               f"took {full * 1e3:.0f} ms")
-    return {"impl": "reference",
-            "metric": "decode qgemv weight GB/s (% of HBM peak); prefill qgemm TFLOP/s (% peak)",
+    return {"impl": "reference", "metric": METRIC,
             "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": sec * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -693,19 +917,16 @@ def run_reference(args, world, rank, budget_s=90.0):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=28000)
+    ap.add_argument("--steps", type=int, default=2800)
     ap.add_argument("--warmup", type=int, default=280)
     ap.add_argument("--impl", default="woq", choices=["woq", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--prefill-m", type=int, default=512)
-    ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--unfused", action="store_true", help="7 launches per block instead of 4")
     ap.add_argument("--m", type=int, default=1, help="activation rows per decode step (1..64)")
     ap.add_argument("--no-lm-head", action="store_true")
     ap.add_argument("--no-fused-epilogues", action="store_true")
-    ap.add_argument("--batched-m", type=int, default=64,
-                    help="rows of the batched-decode leg (qgemm auto path); <= 1 skips it")
+    ap.add_argument("--no-batched", action="store_true", help="skip the M=64 / M=4096 legs")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -720,25 +941,48 @@ def main(argv=None):
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
+    import weight_only_bit_qgemv_b200 as woq
+
     peaks, peak_kind = load_peaks()
-    out, layers, groups, xs = run_decode(args, world, rank, local, peaks, peak_kind)
     device = torch.device("cuda", local)
+    flush = L2Flush(device)
+    stream = torch.cuda.Stream(device)
+    out, layers, groups, xs = run_decode(args, world, local, peaks, peak_kind, flush)
+    configs = {"decoder_block_m1": {"workload": out["config"]["workload"], "dtype": "f32",
+                                    "gbs": out["value"], "us_per_step": round(out["ms_per_step"] * 1e3, 3),
+                                    "roofline": out["roofline"], "note": "the headline line itself"}}
+    configs["single_qgemv_m1"] = run_single_qgemv(device, peaks, peak_kind, stream, world, flush)
+    lm8 = None
     if not args.no_lm_head:
-        out["kernel_roofline_lm_head"] = run_lm_head_roofline(device, peaks, peak_kind)
+        configs["lm_head_m1_int8"] = run_lm_head(device, peaks, peak_kind, 8)
+        configs["lm_head_m1_int4"] = run_lm_head(device, peaks, peak_kind, 4)
+        n, k = workloads.LM_HEAD
+        lm8 = woq.pack(workloads.weight(n, k, seed=workloads.LM_HEAD_SEED), 8, device)
     if not args.no_prefill:
-        out["prefill"] = run_prefill(layers, groups, device, args.prefill_m, 3, peaks, peak_kind,
-                                     world)
-    if args.batched_m > 1:
-        out["batched_decode"] = run_batched_decode(layers, groups, device, args.batched_m,
-                                                   280, peaks, peak_kind, world)
+        configs["prefill_m512"] = run_prefill(layers, groups, device, 512, peaks, peak_kind,
+                                              stream, world, flush)
+    if not args.no_batched:
+        configs["decoder_m64_plus_lm_head"] = run_batched_decode(
+            layers, groups, device, 64, peaks, peak_kind, stream, world, flush, lm_head=lm8)
+        if not args.no_prefill:
+            configs["prefill_m4096_plus_lm_head"] = run_prefill(
+                layers, groups, device, 4096, peaks, peak_kind, stream, world, flush, lm_head=lm8)
     if not args.no_fused_epilogues:
-        fe = run_fused_epilogues(layers, groups, device, 2800, world)
+        fe = run_fused_epilogues(layers, groups, device, stream, world, flush)
         if fe is not None:
             out["fused_epilogues"] = fe
-    if rank == 0 and not args.no_cpu_baseline and args.m == 1:
-        cb, parity = cpu_baseline_leg(layers[0], groups, xs, args.cpu_budget)
-        out["cpu_baseline"] = cb
+    if rank == 0 and not args.no_cpu_baseline and args.m == 1 and not args.unfused:
+        legs, parity = cpu_legs(groups, layers[0], xs)
+        out["cpu_baseline"] = legs.pop("decoder_block_m1")
         out["parity"] = parity
+        configs["decoder_block_m1"]["cpu_baseline"] = out["cpu_baseline"]
+        key_of = {"single_qgemv_m1": "single_qgemv_m1", "lm_head_m1_int8": "lm_head_m1_int8",
+                  "prefill_m512": "prefill_m512", "decoder_m64": "decoder_m64_plus_lm_head",
+                  "prefill_m4096": "prefill_m4096_plus_lm_head"}
+        for leg, cfg in key_of.items():
+            if cfg in configs:
+                configs[cfg]["cpu_baseline"] = legs[leg]
+    out["configs"] = configs
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

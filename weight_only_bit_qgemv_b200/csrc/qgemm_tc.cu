@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kTmemCols = 2 * kAccCols;   // two accumulator sets
   static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
   constexpr uint32_t kIdesc = idesc_for(kAccCols);
+  constexpr uint32_t kIdescLo = idesc_for(SPLIT ? TM : kAccCols);  // split form: x hi rows only
   const Layout L = make_layout(BITS, BN, kAStage, kBBytes, kSB, sx_stages, sw_stages, sc_bytes, sc_bufs);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -431,8 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (ks != ks0 || kk != 0) ? 1u : 0u;
             if constexpr (SPLIT) {
+              // weight hi against x hi and x lo (N = 128); weight lo against x hi only
+              // (N = 64, the first 64 X tile rows): the dropped lo x lo product is below
+              // 2^-16 of each term.
               ptx::tc_mma_f16(d, bd + 2 * kk, ad + 2 * kk, kIdesc, acc);
-              ptx::tc_mma_f16(d, bd + (kBBytes1 >> 4) + 2 * kk, ad + 2 * kk, kIdesc, 1u);
+              ptx::tc_mma_f16(d, bd + (kBBytes1 >> 4) + 2 * kk, ad + 2 * kk, kIdescLo, 1u);
             } else if constexpr (MH == 2) {
               ptx::tc_mma_f16(d, bd + 2 * kk, ad + 2 * kk, kIdesc, acc);
             } else {
@@ -600,23 +604,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t *xs = smem + L.a + s * kAStage;
-        for (int job = et; job < rows * 8; job += kEpiWarps * 32) {
+        // A stage is at most TM * 8 = 512 jobs of 8 values, four per epilogue thread: all of a
+        // thread's loads are issued before any is used, so a stage costs one L2 round trip.
+        constexpr int kJobsPerThread = TM * 8 / (kEpiWarps * 32);
+        float4 va[kJobsPerThread], vb[kJobsPerThread];
+#pragma unroll
+        for (int i = 0; i < kJobsPerThread; ++i) {
+          const int job = et + i * kEpiWarps * 32;
           const int r = job >> 3, c = job & 7;
           const int col = ks * BK + c * 8;
-          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-          if (col < K) {
+          va[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          vb[i] = va[i];
+          if (r < rows && col < K) {
             const float4 *src = reinterpret_cast<const float4 *>(xt + static_cast<size_t>(r) * K + col);
-            a = __ldg(src);
-            b = __ldg(src + 1);
+            va[i] = __ldg(src);
+            vb[i] = __ldg(src + 1);
           }
-          uint4 h, l;
-          split_pack(a.x, a.y, h.x, l.x);
-          split_pack(a.z, a.w, h.y, l.y);
-          split_pack(b.x, b.y, h.z, l.z);
-          split_pack(b.z, b.w, h.w, l.w);
-          const int off = (c ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4 *>(xs + r * 128 + off) = h;
-          *reinterpret_cast<uint4 *>(xs + (TM + r) * 128 + off) = l;
+        }
+#pragma unroll
+        for (int i = 0; i < kJobsPerThread; ++i) {
+          const int job = et + i * kEpiWarps * 32;
+          const int r = job >> 3, c = job & 7;
+          if (r < rows) {
+            uint4 h, l;
+            split_pack(va[i].x, va[i].y, h.x, l.x);
+            split_pack(va[i].z, va[i].w, h.y, l.y);
+            split_pack(vb[i].x, vb[i].y, h.z, l.z);
+            split_pack(vb[i].z, vb[i].w, h.w, l.w);
+            const int off = (c ^ (r & 7)) << 4;
+            *reinterpret_cast<uint4 *>(xs + r * 128 + off) = h;
+            *reinterpret_cast<uint4 *>(xs + (TM + r) * 128 + off) = l;
+          }
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
