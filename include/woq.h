@@ -125,14 +125,27 @@ int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream
  *                       significand bits; error stays within the FP32 tolerance of qgemv.
  *                       Needs 2 <= m <= 64, k % 256 == 0 and k <= 8192, else WOQ_ESHAPE.
  *   WOQ_GEMV_SPLIT_GEMM the tcgen05 split GEMM of qgemm's WOQ_PATH_SPLIT_TC (x and s*q each
- *                       as bf16 hi + lo, all four products in an FP32 tensor-memory
- *                       accumulator, 64-row tiles); no workspace. Any 1 <= m <= 64.
+ *                       as bf16 hi + lo, products in an FP32 tensor-memory accumulator,
+ *                       64-row tiles); no workspace. Any 1 <= m <= 64.
+ *   WOQ_GEMV_INT8_TC    the integer tensor cores (tcgen05 kind::i8), following
+ *                       "TinyMOSS-Diarize", "What's next" (an i8mm path that does not quantise
+ *                       the activations): per activation row and 32-block, x is written
+ *                       exactly enough as 2^E (d0 + d1 2^-7 + d2 2^-14) with integer digits
+ *                       |d_i| <= 64 and the block's own power-of-two exponent E (remainder
+ *                       below 2^-20 of the block's largest |x|); the codes (int8 as they are,
+ *                       int4 times 16) are multiplied by each digit exactly in int32, one sum
+ *                       per block, and the block sums are scaled by 2^E and the binary16 scale
+ *                       and accumulated in FP32. K-splits of a 128-row tile run as one
+ *                       thread-block cluster and are summed in shared memory in a fixed order.
+ *                       Needs 1 <= m <= 4 and k % 128 == 0, else WOQ_ESHAPE. A block holding a
+ *                       non-finite x makes the outputs it feeds NaN.
  * Arguments and errors otherwise as qgemv; an unknown path is WOQ_EINVAL.
  */
 #define WOQ_GEMV_AUTO       0
 #define WOQ_GEMV_CUDA_CORE  1
 #define WOQ_GEMV_SPLIT_TC   2
 #define WOQ_GEMV_SPLIT_GEMM 3
+#define WOQ_GEMV_INT8_TC    4
 int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t path,
                void *stream);
 

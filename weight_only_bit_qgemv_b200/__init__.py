@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     WOQ_GEMV_CUDA_CORE,
     WOQ_GEMV_SPLIT_TC,
     WOQ_GEMV_SPLIT_GEMM,
+    WOQ_GEMV_INT8_TC,
     WOQ_PATH_AUTO,
     WOQ_PATH_BF16_TC,
     WOQ_PATH_FP32,
@@ -57,6 +58,7 @@ _GEMV_PATHS = {
     "cuda_core": WOQ_GEMV_CUDA_CORE,
     "split_tc": WOQ_GEMV_SPLIT_TC,
     "split_gemm": WOQ_GEMV_SPLIT_GEMM,
+    "int8_tc": WOQ_GEMV_INT8_TC,
 }
 
 
@@ -121,7 +123,7 @@ def qgemv(
     path: str = "auto",
 ) -> torch.Tensor:
     """y[m, n] = x[m, k] . W_hat^T, 1 <= m <= 64, FP32 accuracy (C ABI ``qgemv_path``);
-    path in {"auto", "cuda_core", "split_tc", "split_gemm"}."""
+    path in {"auto", "cuda_core", "split_tc", "split_gemm", "int8_tc"}."""
     if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
         raise ValueError("x must be a contiguous 2-D float32 CUDA tensor")
     m = x.shape[0]

@@ -26,6 +26,7 @@ WOQ_GEMV_AUTO = 0
 WOQ_GEMV_CUDA_CORE = 1
 WOQ_GEMV_SPLIT_TC = 2
 WOQ_GEMV_SPLIT_GEMM = 3
+WOQ_GEMV_INT8_TC = 4
 
 #: Every symbol include/woq.h declares.
 EXPORTS = (

@@ -13,7 +13,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libwoq.so")
 
-CU_SOURCES = ["api.cu", "qgemv.cu", "qgemv_tc.cu", "qgemm_tc.cu", "qgemm_noalloc.cu"]
+CU_SOURCES = ["api.cu", "qgemv.cu", "qgemv_tc.cu", "qgemv_i8tc.cu", "qgemm_tc.cu", "qgemm_noalloc.cu"]
 CXX_SOURCES = ["qpack.cpp"]
 HEADERS = ["ptx.cuh", "woq_internal.h"]
 

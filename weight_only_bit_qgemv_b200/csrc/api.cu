@@ -81,7 +81,7 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
   if (!x || !y) return WOQ_EINVAL;
   if (m < 1 || m > 64) return WOQ_EINVAL;
   if (path != WOQ_GEMV_AUTO && path != WOQ_GEMV_CUDA_CORE && path != WOQ_GEMV_SPLIT_TC &&
-      path != WOQ_GEMV_SPLIT_GEMM)
+      path != WOQ_GEMV_SPLIT_GEMM && path != WOQ_GEMV_INT8_TC)
     return WOQ_EINVAL;
   if (w->k > 32768) return WOQ_ESHAPE;
   if (!woq::aligned(x, 16) || !woq::aligned(y, 16)) return WOQ_EALIGN;
@@ -89,6 +89,10 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
   rc = woq::current_device(&dev);
   if (rc != WOQ_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (path == WOQ_GEMV_INT8_TC) {
+    rc = woq::launch_gemv_i8tc(x, m, *w, y, s, dev);
+    return rc == 1 ? WOQ_ESHAPE : rc;
+  }
   const bool wide = (w->n + 127) / 128 >= dev.sm_count;
   if (path == WOQ_GEMV_SPLIT_GEMM ||
       (path == WOQ_GEMV_AUTO && m >= (wide ? kGemmMinMWide : kGemmMinM))) {
@@ -213,14 +217,16 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
 
 int woq_device_status(int clear) {
   if (cudaDeviceSynchronize() != cudaSuccess) return WOQ_ECUDA;
-  unsigned v = 0, g = 0, t = 0;
+  unsigned v = 0, g = 0, t = 0, i = 0;
   int rc = woq::read_wait_timeout_flag(clear, &v);
   if (rc != WOQ_OK) return rc;
   rc = woq::read_gemv_timeout_flag(clear, &g);
   if (rc != WOQ_OK) return rc;
   rc = woq::read_gemv_tc_timeout_flag(clear, &t);
   if (rc != WOQ_OK) return rc;
-  return (v || g || t) ? WOQ_ETIMEOUT : WOQ_OK;
+  rc = woq::read_i8tc_timeout_flag(clear, &i);
+  if (rc != WOQ_OK) return rc;
+  return (v || g || t || i) ? WOQ_ETIMEOUT : WOQ_OK;
 }
 
 void woq_debug_set_wait_limit(long long cycles) { woq::set_wait_limit_cycles(cycles); }

@@ -56,6 +56,13 @@ int launch_gemv_tc(const float *x, int64_t m, const woq_weight &w, float *y, cud
                    const DevInfo &dev);
 int read_gemv_tc_timeout_flag(int clear, unsigned *value);
 
+// ---- qgemv_i8tc.cu ----
+// Small-batch GEMV on the integer tensor cores (1 <= m <= 4; x as three signed digits per
+// 32-block, exact int32 block sums). Returns 1 (nothing launched) for shapes it does not take.
+int launch_gemv_i8tc(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                     const DevInfo &dev);
+int read_i8tc_timeout_flag(int clear, unsigned *value);
+
 // ---- qgemm_tc.cu ----
 // How the tensor-core path runs a problem: tile width, K-splits and workspace layout
 // ([bf16 copy of X][FP32 partials of the splits], each 256-byte aligned).
