@@ -64,7 +64,7 @@ def test_argument_checks_return_before_touching_a_device():
     assert L.qgemv(ok_ptr + 4, 1, ctypes.byref(w), ok_ptr, None) == _lib.WOQ_EALIGN
     big = _w(k=65536, packed=ok_ptr, scales=ok_ptr)
     assert L.qgemv(ok_ptr, 1, ctypes.byref(big), ok_ptr, None) == _lib.WOQ_ESHAPE
-    assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, 4, None) == _lib.WOQ_EINVAL
+    assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, 5, None) == _lib.WOQ_EINVAL
     assert L.qgemv_path(ok_ptr, 8, ctypes.byref(w), ok_ptr, -1, None) == _lib.WOQ_EINVAL
     assert L.qgemv_path(ok_ptr, 65, ctypes.byref(w), ok_ptr, _lib.WOQ_GEMV_SPLIT_TC, None) == _lib.WOQ_EINVAL
     # qgemv_swiglu: 1 <= m <= 64, n even
