@@ -201,6 +201,46 @@ int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, f
                  void *stream);
 
 /*
+ * qgemv_chain -- a decode step's GEMVs as one persistent launch, in order ("TinyMOSS-Diarize",
+ * "What we learned": match the threading granularity to the size of the operation; a decoder
+ * block's projections at one token are each too small to fill the GPU). Item i computes
+ *   WOQ_EPI_NONE      y = x . W_hat^T                         y [m, n]
+ *   WOQ_EPI_SWIGLU    y[j, i] = silu(g) * u over rows 2i (gate), 2i+1 (up), as qgemv_swiglu
+ *                                                             y [m, n/2]
+ *   WOQ_EPI_RESIDUAL  y = x . W_hat^T + r, r may be y itself  y [m, n]
+ * with the arithmetic of qgemv's CUDA-core form (exact codes, each 32-block's FP32 sum scaled
+ * once by its binary16 scale, FP32 accumulation; when a row's K is split across warps, the
+ * parts are added in a fixed order). Item i reads its x (and r) only after every earlier
+ * item's outputs are complete, so an input may be an earlier item's output: the launch keeps
+ * the order that separate calls on one stream would have. Deterministic.
+ *   items     host array of `count` descriptors (read during the call only), 1 <= count <= 8
+ *   m         activation rows, 1 <= m <= 8
+ *   workspace device, 256-byte aligned, >= qgemv_chain_workspace_bytes() bytes: counters that
+ *             must be zero before the first call; every call that returns WOQ_OK leaves them
+ *             zero again (after a WOQ_ETIMEOUT from woq_device_status, zero them before reuse).
+ *             Calls sharing one workspace must be ordered on one stream.
+ * Each item: w as for qgemv with k % 256 == 0 and k <= 8192; x [m, k] and y device, 16-byte
+ * aligned, y not overlapping x; r (WOQ_EPI_RESIDUAL only) device, 16-byte aligned, equal to y
+ * or not overlapping it. Errors: WOQ_EINVAL, WOQ_ESHAPE, WOQ_EALIGN, WOQ_EWORKSPACE,
+ * WOQ_EDEVICE, WOQ_ECUDA. The launch holds one CTA per SM, and its CTAs wait for one another
+ * between items (bounded waits: a wait that gives up is reported by woq_device_status).
+ */
+#define WOQ_EPI_NONE       0
+#define WOQ_EPI_SWIGLU     1
+#define WOQ_EPI_RESIDUAL   2
+#define WOQ_CHAIN_MAX_ITEMS 8
+typedef struct woq_chain_item {
+  const woq_weight *w;
+  const float *x;
+  float *y;
+  const float *r;
+  int32_t epilogue;
+} woq_chain_item;
+size_t qgemv_chain_workspace_bytes(void);
+int qgemv_chain(const woq_chain_item *items, int32_t count, int64_t m, void *workspace,
+                size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of device workspace qgemm needs for (m, w, path); 0 if none. Returns 0 for
  * invalid arguments too (qgemm itself reports those).
  */
@@ -271,8 +311,11 @@ int qgemm_bf16_noalloc(const float *X, int64_t m, const woq_weight *w, float *Y,
 int woq_device_status(int clear);
 
 /*
- * woq_debug_set_wait_limit -- test hook for the tensor-core qgemm kernel's bounded waits,
- * applied to launches that follow. cycles > 0 sets the cycle budget of every wait;
+ * woq_debug_set_wait_limit -- test hook for the bounded waits of the tensor-core qgemm kernel
+ * and of qgemv_chain, applied to launches that follow. cycles > 0 sets the cycle budget of
+ * every wait (qgemv_chain: of its waits for weights and for the other CTAs); in qgemv_chain,
+ * cycles < 0 makes each CTA's waits for the other CTAs wait for one arrival more than there
+ * are CTAs, bounded by -cycles cycles, so they give up deterministically;
  * 0 restores the default (2^32 cycles, about two seconds); cycles < 0 keeps the default
  * and makes the MMA-issuing thread of every CTA first wait on a barrier that nothing
  * arrives on, bounded by -cycles cycles, so the give-up path runs deterministically

@@ -40,6 +40,9 @@ __all__ = [
     "qgemv_swiglu",
     "qgemv_residual",
     "interleave_rows",
+    "ChainItem",
+    "chain_workspace",
+    "qgemv_chain",
     "qgemm",
     "qgemm_workspace_bytes",
     "device_status",
@@ -184,6 +187,49 @@ def qgemv_residual(x: torch.Tensor, w: PackedWeight, r: torch.Tensor, out: torch
     rc = _lib.lib().qgemv_residual(_ptr(x), m, ctypes.byref(d), _ptr(r), _ptr(out), _stream(stream))
     _lib.check(rc, "qgemv_residual")
     return out
+
+
+_EPILOGUES = {"none": _lib.WOQ_EPI_NONE, "swiglu": _lib.WOQ_EPI_SWIGLU, "residual": _lib.WOQ_EPI_RESIDUAL}
+
+
+@dataclass
+class ChainItem:
+    """One GEMV of a qgemv_chain launch: y = x . W_hat^T, with epilogue "none", "swiglu" (rows
+    interleaved gate/up; y [m, n/2]) or "residual" (y = ... + r, r may be y)."""
+
+    w: PackedWeight
+    x: torch.Tensor
+    y: torch.Tensor
+    r: torch.Tensor | None = None
+    epilogue: str = "none"
+
+
+def chain_workspace(device="cuda") -> torch.Tensor:
+    """A zeroed workspace for qgemv_chain (its counters; every successful call leaves them zero)."""
+    return torch.zeros(int(_lib.lib().qgemv_chain_workspace_bytes()), dtype=torch.uint8, device=device)
+
+
+def qgemv_chain(items: list[ChainItem], workspace: torch.Tensor, stream=None) -> None:
+    """Run the items in order as one persistent launch (C ABI ``qgemv_chain``); item i reads
+    its x only after every earlier item's outputs are complete."""
+    if not items:
+        raise ValueError("qgemv_chain needs at least one item")
+    m = items[0].x.shape[0]
+    descs = [it.w.desc() for it in items]  # kept alive for the call
+    arr = (_lib.WoqChainItem * len(items))()
+    for i, (it, d) in enumerate(zip(items, descs)):
+        for t in (it.x, it.y) + ((it.r,) if it.r is not None else ()):
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError("chain tensors must be contiguous float32 CUDA tensors")
+        if it.x.shape[0] != m:
+            raise ValueError("every item must have the same number of activation rows")
+        arr[i].w = ctypes.pointer(d)
+        arr[i].x = _ptr(it.x)
+        arr[i].y = _ptr(it.y)
+        arr[i].r = _ptr(it.r) if it.r is not None else None
+        arr[i].epilogue = _EPILOGUES[it.epilogue]
+    rc = _lib.lib().qgemv_chain(arr, len(items), m, _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(rc, "qgemv_chain")
 
 
 def qgemm_workspace_bytes(m: int, w: PackedWeight, path: str = "auto") -> int:

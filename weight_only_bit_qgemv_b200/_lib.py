@@ -27,6 +27,10 @@ WOQ_GEMV_CUDA_CORE = 1
 WOQ_GEMV_SPLIT_TC = 2
 WOQ_GEMV_SPLIT_GEMM = 3
 WOQ_GEMV_INT8_TC = 4
+WOQ_EPI_NONE = 0
+WOQ_EPI_SWIGLU = 1
+WOQ_EPI_RESIDUAL = 2
+WOQ_CHAIN_MAX_ITEMS = 8
 
 #: Every symbol include/woq.h declares.
 EXPORTS = (
@@ -36,6 +40,8 @@ EXPORTS = (
     "qgemv_swiglu",
     "qgemv_residual",
     "qgemv_argmax",
+    "qgemv_chain_workspace_bytes",
+    "qgemv_chain",
     "qgemm_workspace_bytes",
     "qgemm",
     "qgemm_bf16_noalloc",
@@ -55,6 +61,16 @@ class WoqWeight(ctypes.Structure):
         ("k", ctypes.c_int64),
         ("packed", ctypes.c_void_p),
         ("scales", ctypes.c_void_p),
+    ]
+
+
+class WoqChainItem(ctypes.Structure):
+    _fields_ = [
+        ("w", ctypes.POINTER(WoqWeight)),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("r", ctypes.c_void_p),
+        ("epilogue", ctypes.c_int32),
     ]
 
 
@@ -92,6 +108,10 @@ def lib() -> ctypes.CDLL:
     L.qgemv_residual.restype = ctypes.c_int
     L.qgemv_argmax.argtypes = [vp, c_i64, wp, vp, vp, vp]
     L.qgemv_argmax.restype = ctypes.c_int
+    L.qgemv_chain_workspace_bytes.argtypes = []
+    L.qgemv_chain_workspace_bytes.restype = ctypes.c_size_t
+    L.qgemv_chain.argtypes = [ctypes.POINTER(WoqChainItem), c_i32, c_i64, vp, ctypes.c_size_t, vp]
+    L.qgemv_chain.restype = ctypes.c_int
     L.qgemm_workspace_bytes.argtypes = [c_i64, wp, c_i32]
     L.qgemm_workspace_bytes.restype = ctypes.c_size_t
     L.qgemm.argtypes = [vp, c_i64, wp, vp, c_i32, vp, ctypes.c_size_t, vp]

@@ -13,9 +13,9 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libwoq.so")
 
-CU_SOURCES = ["api.cu", "qgemv.cu", "qgemv_tc.cu", "qgemv_i8tc.cu", "qgemm_tc.cu", "qgemm_noalloc.cu"]
+CU_SOURCES = ["api.cu", "qgemv.cu", "qgemv_tc.cu", "qgemv_i8tc.cu", "qgemv_chain.cu", "qgemm_tc.cu", "qgemm_noalloc.cu"]
 CXX_SOURCES = ["qpack.cpp"]
-HEADERS = ["ptx.cuh", "woq_internal.h"]
+HEADERS = ["ptx.cuh", "woq_internal.h", "gemv_math.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -157,6 +157,44 @@ int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, f
   return woq::launch_gemv_argmax(x, m, *w, idx, val, static_cast<cudaStream_t>(stream), dev);
 }
 
+size_t qgemv_chain_workspace_bytes(void) { return 256; }
+
+int qgemv_chain(const woq_chain_item *items, int32_t count, int64_t m, void *workspace,
+                size_t workspace_bytes, void *stream) {
+  if (!items || count < 1 || count > WOQ_CHAIN_MAX_ITEMS) return WOQ_EINVAL;
+  if (m < 1 || m > 8) return WOQ_EINVAL;
+  if (!workspace || workspace_bytes < qgemv_chain_workspace_bytes()) return WOQ_EWORKSPACE;
+  if (!woq::aligned(workspace, 256)) return WOQ_EALIGN;
+  auto overlap = [](const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+  };
+  for (int32_t i = 0; i < count; ++i) {
+    const woq_chain_item &it = items[i];
+    int rc = woq::check_weight(it.w);
+    if (rc != WOQ_OK) return rc;
+    if (!it.x || !it.y) return WOQ_EINVAL;
+    if (it.epilogue != WOQ_EPI_NONE && it.epilogue != WOQ_EPI_SWIGLU && it.epilogue != WOQ_EPI_RESIDUAL)
+      return WOQ_EINVAL;
+    if (it.w->k % 256 != 0 || it.w->k > 8192) return WOQ_ESHAPE;
+    if (it.epilogue == WOQ_EPI_SWIGLU && it.w->n % 2 != 0) return WOQ_ESHAPE;
+    if (!woq::aligned(it.x, 16) || !woq::aligned(it.y, 16)) return WOQ_EALIGN;
+    const size_t xb = static_cast<size_t>(m) * it.w->k * 4;
+    const size_t yb = static_cast<size_t>(m) * (it.epilogue == WOQ_EPI_SWIGLU ? it.w->n / 2 : it.w->n) * 4;
+    if (overlap(it.x, xb, it.y, yb)) return WOQ_EINVAL;
+    if (it.epilogue == WOQ_EPI_RESIDUAL) {
+      if (!it.r) return WOQ_EINVAL;
+      if (!woq::aligned(it.r, 16)) return WOQ_EALIGN;
+      if (it.r != it.y && overlap(it.r, yb, it.y, yb)) return WOQ_EINVAL;
+    }
+  }
+  DevInfo dev;
+  int rc = woq::current_device(&dev);
+  if (rc != WOQ_OK) return rc;
+  return woq::launch_gemv_chain(items, count, m, static_cast<unsigned *>(workspace),
+                                static_cast<cudaStream_t>(stream), dev);
+}
+
 // SM count the tensor-core plan is made for: the current device's, or 0 (no K-splits) when
 // no device can be queried, so that sizing never fails.
 static int plan_sm_count() {
@@ -217,7 +255,7 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
 
 int woq_device_status(int clear) {
   if (cudaDeviceSynchronize() != cudaSuccess) return WOQ_ECUDA;
-  unsigned v = 0, g = 0, t = 0, i = 0;
+  unsigned v = 0, g = 0, t = 0, i = 0, c = 0;
   int rc = woq::read_wait_timeout_flag(clear, &v);
   if (rc != WOQ_OK) return rc;
   rc = woq::read_gemv_timeout_flag(clear, &g);
@@ -226,7 +264,9 @@ int woq_device_status(int clear) {
   if (rc != WOQ_OK) return rc;
   rc = woq::read_i8tc_timeout_flag(clear, &i);
   if (rc != WOQ_OK) return rc;
-  return (v || g || t || i) ? WOQ_ETIMEOUT : WOQ_OK;
+  rc = woq::read_chain_timeout_flag(clear, &c);
+  if (rc != WOQ_OK) return rc;
+  return (v || g || t || i || c) ? WOQ_ETIMEOUT : WOQ_OK;
 }
 
 void woq_debug_set_wait_limit(long long cycles) { woq::set_wait_limit_cycles(cycles); }

@@ -1,0 +1,225 @@
+// Exact FP32 arithmetic of the CUDA-core GEMV kernels (qgemv.cu, qgemv_chain.cu): packed
+// int4/int8 codes to exact FP32 values with one LOP3 / PRMT per code, products with staged x
+// rows, one binary16 scale per 32-block applied to the block's sum.
+//
+// Codes become exact FP32 values with a single LOP3 per element: the 4-bit field (offset by
+// 8) is placed in the low mantissa bits of 2^23 and the bias is removed with one exact
+// packed subtraction (f32x2). int4 fields at nibble position j of a 16-bit half carry a
+// factor 2^(4j) that is removed, exactly, once per block.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace woq {
+namespace gemv {
+
+// 16-byte unit u of an x row lives at unit swz(u) in shared memory.
+__device__ __forceinline__ int swz(int u) { return u ^ ((u >> 3) & 7); }
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// One 32-bit word of int4 codes (elements e0..e7, e_p in bits 4p..4p+3) -> four exact
+// pairs p[j] = (q_j, q_{4+j}) * 2^(4j).
+__device__ __forceinline__ void unpack_int4_word(uint32_t w, float2 (&p)[4]) {
+  const uint32_t hi = w >> 16;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t mask = 0xFu << (4 * j);
+    const uint32_t magic = 0x4B000000u | (0x8u << (4 * j));  // 2^23, field offset by 8
+    const float bias = 8388608.0f + 8.0f * static_cast<float>(1u << (4 * j));
+    const float lo_f = __uint_as_float((w & mask) ^ magic);
+    const float hi_f = __uint_as_float((hi & mask) ^ magic);
+    p[j] = __fadd2_rn(make_float2(lo_f, hi_f), make_float2(-bias, -bias));
+  }
+}
+
+// One 32-bit word of int8 codes (elements e0..e3 in bytes 0..3) -> (q0, q1), (q2, q3).
+__device__ __forceinline__ void unpack_int8_word(uint32_t w, float2 (&p)[2]) {
+  const uint32_t u = w ^ 0x80808080u;  // offset binary, q + 128
+  const float bias = 8388608.0f + 128.0f;
+  const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540));
+  const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541));
+  const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542));
+  const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543));
+  p[0] = __fadd2_rn(make_float2(f0, f1), make_float2(-bias, -bias));
+  p[1] = __fadd2_rn(make_float2(f2, f3), make_float2(-bias, -bias));
+}
+
+__device__ __forceinline__ float fold_int4(const float2 (&a)[4]) {
+  float2 t = __ffma2_rn(a[1], make_float2(0.0625f, 0.0625f), a[0]);
+  t = __ffma2_rn(a[2], make_float2(0.00390625f, 0.00390625f), t);
+  t = __ffma2_rn(a[3], make_float2(0.000244140625f, 0.000244140625f), t);
+  return t.x + t.y;
+}
+
+// int4: one 16-byte chunk (one block of 32) of R rows against MT x rows.
+template <int MT, int R>
+__device__ __forceinline__ void chunk_int4(const float4 *__restrict__ xs4, int units_row, int c,
+                                           const uint4 (&wv)[R], const float (&sc)[R],
+                                           float (&acc)[R][MT]) {
+  if constexpr (MT <= 2) {
+    float4 xv[MT][8];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) xv[mm][t] = xs4[mm * units_row + swz(8 * c + t)];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 a2[MT][4];
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a2[mm][j] = make_float2(0.f, 0.f);
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 p[4];
+        unpack_int4_word(ws[i], p);
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          const float4 xa = xv[mm][2 * i], xb = xv[mm][2 * i + 1];
+          a2[mm][0] = __ffma2_rn(p[0], make_float2(xa.x, xa.y), a2[mm][0]);
+          a2[mm][1] = __ffma2_rn(p[1], make_float2(xa.z, xa.w), a2[mm][1]);
+          a2[mm][2] = __ffma2_rn(p[2], make_float2(xb.x, xb.y), a2[mm][2]);
+          a2[mm][3] = __ffma2_rn(p[3], make_float2(xb.z, xb.w), a2[mm][3]);
+        }
+      }
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], fold_int4(a2[mm]), acc[r][mm]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 p[4][4];
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) unpack_int4_word(ws[i], p[i]);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float2 a2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 xa = xs4[mm * units_row + swz(8 * c + 2 * i)];
+          const float4 xb = xs4[mm * units_row + swz(8 * c + 2 * i + 1)];
+          a2[0] = __ffma2_rn(p[i][0], make_float2(xa.x, xa.y), a2[0]);
+          a2[1] = __ffma2_rn(p[i][1], make_float2(xa.z, xa.w), a2[1]);
+          a2[2] = __ffma2_rn(p[i][2], make_float2(xb.x, xb.y), a2[2]);
+          a2[3] = __ffma2_rn(p[i][3], make_float2(xb.z, xb.w), a2[3]);
+        }
+        acc[r][mm] = fmaf(sc[r], fold_int4(a2), acc[r][mm]);
+      }
+    }
+  }
+}
+
+// int8: one 16-byte chunk (half a block) of R rows against MT x rows.
+template <int MT, int R>
+__device__ __forceinline__ void chunk_int8(const float4 *__restrict__ xs4, int units_row, int c,
+                                           const uint4 (&wv)[R], const float (&sc)[R],
+                                           float (&acc)[R][MT]) {
+  if constexpr (MT <= 2) {
+    float4 xv[MT][4];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) xv[mm][t] = xs4[mm * units_row + swz(4 * c + t)];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 a2[MT];
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) a2[mm] = make_float2(0.f, 0.f);
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 p[2];
+        unpack_int8_word(ws[i], p);
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          a2[mm] = __ffma2_rn(p[0], make_float2(xv[mm][i].x, xv[mm][i].y), a2[mm]);
+          a2[mm] = __ffma2_rn(p[1], make_float2(xv[mm][i].z, xv[mm][i].w), a2[mm]);
+        }
+      }
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], a2[mm].x + a2[mm].y, acc[r][mm]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 p[4][2];
+      const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) unpack_int8_word(ws[i], p[i]);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 xa = xs4[mm * units_row + swz(4 * c + i)];
+          a2 = __ffma2_rn(p[i][0], make_float2(xa.x, xa.y), a2);
+          a2 = __ffma2_rn(p[i][1], make_float2(xa.z, xa.w), a2);
+        }
+        acc[r][mm] = fmaf(sc[r], a2.x + a2.y, acc[r][mm]);
+      }
+    }
+  }
+}
+
+// int8: one whole block (32 codes = chunks 2b and 2b+1, x units 8b .. 8b+7) of R rows
+// against MT x rows; one scale per row, applied once to the block sum.
+template <int MT, int R>
+__device__ __forceinline__ void block_int8(const float4 *__restrict__ xs4, int units_row, int b,
+                                           const uint4 (&lo)[R], const uint4 (&hi)[R],
+                                           const float (&sc)[R], float (&acc)[R][MT]) {
+  if constexpr (MT <= 2) {
+    float4 xv[MT][8];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) xv[mm][t] = xs4[mm * units_row + swz(8 * b + t)];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 a2[MT];
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) a2[mm] = make_float2(0.f, 0.f);
+      const uint32_t ws[8] = {lo[r].x, lo[r].y, lo[r].z, lo[r].w, hi[r].x, hi[r].y, hi[r].z, hi[r].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float2 p[2];
+        unpack_int8_word(ws[i], p);
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          a2[mm] = __ffma2_rn(p[0], make_float2(xv[mm][i].x, xv[mm][i].y), a2[mm]);
+          a2[mm] = __ffma2_rn(p[1], make_float2(xv[mm][i].z, xv[mm][i].w), a2[mm]);
+        }
+      }
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], a2[mm].x + a2[mm].y, acc[r][mm]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float2 p[8][2];
+      const uint32_t ws[8] = {lo[r].x, lo[r].y, lo[r].z, lo[r].w, hi[r].x, hi[r].y, hi[r].z, hi[r].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) unpack_int8_word(ws[i], p[i]);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 xa = xs4[mm * units_row + swz(8 * b + i)];
+          a2 = __ffma2_rn(p[i][0], make_float2(xa.x, xa.y), a2);
+          a2 = __ffma2_rn(p[i][1], make_float2(xa.z, xa.w), a2);
+        }
+        acc[r][mm] = fmaf(sc[r], a2.x + a2.y, acc[r][mm]);
+      }
+    }
+  }
+}
+
+}  // namespace gemv
+}  // namespace woq

@@ -63,6 +63,12 @@ int launch_gemv_i8tc(const float *x, int64_t m, const woq_weight &w, float *y, c
                      const DevInfo &dev);
 int read_i8tc_timeout_flag(int clear, unsigned *value);
 
+// ---- qgemv_chain.cu ----
+// A decode step's GEMV items as one persistent launch (arguments already validated).
+int launch_gemv_chain(const woq_chain_item *items, int count, int64_t m, unsigned *counters,
+                      cudaStream_t s, const DevInfo &dev);
+int read_chain_timeout_flag(int clear, unsigned *value);
+
 // ---- qgemm_tc.cu ----
 // How the tensor-core path runs a problem: tile width, K-splits and workspace layout
 // ([bf16 copy of X][FP32 partials of the splits], each 256-byte aligned).
@@ -84,7 +90,9 @@ int launch_gemm_tc(const float *X, int64_t m, const woq_weight &w, float *Y, voi
 // Reads (and optionally clears) the device-side record of bounded waits that gave up on
 // the current device. Synchronous.
 int read_wait_timeout_flag(int clear, unsigned *value);
-// Test hook: cycle budget of every bounded wait in the tensor-core kernel (0 = default).
+// Test hook: cycle budget of every bounded wait in the tensor-core kernel and the chained
+// GEMV (0 = default); wait_limit_cycles() reads it back.
 void set_wait_limit_cycles(long long cycles);
+long long wait_limit_cycles();
 
 }  // namespace woq
