@@ -106,16 +106,6 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   return v;
 }
 
-// The same load without a memory clobber, so that several can be in flight at once; it stays
-// ordered after a preceding cluster barrier (both are volatile asm).
-__device__ __forceinline__ float4 ld_shared_cluster_v4_async(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr));
-  return v;
-}
-
 // ---- fences ----------------------------------------------------------------------------
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor-core operand reads, bulk copies).

@@ -595,11 +595,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // never read.
     {
       const float *xt = Xf + static_cast<size_t>(mb * TM) * K;
-      // A stage is at most TM * 8 = 512 jobs of 8 values, four per epilogue thread. The loads
-      // of the next stage are issued before this stage is converted and stored (they read
-      // global X, not the slot), so the stages' L2 round trips overlap.
-      constexpr int kJobsPerThread = TM * 8 / (kEpiWarps * 32);
-      auto load_stage = [&](int ks, float4 (&va)[kJobsPerThread], float4 (&vb)[kJobsPerThread]) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ks = ks0; ks < ks1 && ok; ++ks) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.xempty[s], ph ^ 1, wait_limit, abort))) {
+          record_timeout(abort);
+          ok = false;
+          break;
+        }
+        uint8_t *xs = smem + L.a + s * kAStage;
+        // A stage is at most TM * 8 = 512 jobs of 8 values, four per epilogue thread: all of a
+        // thread's loads are issued before any is used, so a stage costs one L2 round trip.
+        constexpr int kJobsPerThread = TM * 8 / (kEpiWarps * 32);
+        float4 va[kJobsPerThread], vb[kJobsPerThread];
 #pragma unroll
         for (int i = 0; i < kJobsPerThread; ++i) {
           const int job = et + i * kEpiWarps * 32;
@@ -613,20 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             vb[i] = __ldg(src + 1);
           }
         }
-      };
-      float4 va[kJobsPerThread], vb[kJobsPerThread];
-      if (ks0 < ks1) load_stage(ks0, va, vb);
-      int s = 0;
-      uint32_t ph = 0;
-      for (int ks = ks0; ks < ks1 && ok; ++ks) {
-        float4 na[kJobsPerThread], nb[kJobsPerThread];
-        if (ks + 1 < ks1) load_stage(ks + 1, na, nb);
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.xempty[s], ph ^ 1, wait_limit, abort))) {
-          record_timeout(abort);
-          ok = false;
-          break;
-        }
-        uint8_t *xs = smem + L.a + s * kAStage;
 #pragma unroll
         for (int i = 0; i < kJobsPerThread; ++i) {
           const int job = et + i * kEpiWarps * 32;
@@ -648,11 +642,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++s == SX) {
           s = 0;
           ph ^= 1;
-        }
-#pragma unroll
-        for (int i = 0; i < kJobsPerThread; ++i) {
-          va[i] = na[i];
-          vb[i] = nb[i];
         }
       }
     }
@@ -799,20 +788,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = threadIdx.x; i < (j1 - j0) * (BN / 4); i += kThreads) {
         const int j = j0 + i / (BN / 4), c4 = i % (BN / 4);
         const uint32_t off = static_cast<uint32_t>((j * BN + 4 * c4) * 4);
-        // every rank's partial in flight at once, then summed in rank order
-        float4 v[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-          if (r < splits) v[r] = ptx::ld_shared_cluster_v4_async(ptx::mapa_shared(st + off, r));
-        float4 acc = v[0];
-#pragma unroll
-        for (int r = 1; r < 8; ++r) {
-          if (r < splits) {
-            acc.x += v[r].x;
-            acc.y += v[r].y;
-            acc.z += v[r].z;
-            acc.w += v[r].w;
-          }
+        float4 acc = ptx::ld_shared_cluster_v4(ptx::mapa_shared(st + off, 0));
+        for (int r = 1; r < splits; ++r) {
+          const float4 v = ptx::ld_shared_cluster_v4(ptx::mapa_shared(st + off, r));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
         }
         const int n = nb * BN + 4 * c4;
         float *yr = Y + static_cast<size_t>(mb * TM + j) * N + n;
