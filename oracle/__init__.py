@@ -16,6 +16,8 @@ fixtures under ``tests/golden/``). No function here is "parity unpinned".
 from .woq_ref import (  # noqa: F401
     BLOCK,
     qrange,
+    int5_high_bit_position,
+    row_bytes,
     fp16_round,
     fp16_bits_to_float,
     quantise,

@@ -15,6 +15,9 @@ What the method computes, and where it is stated:
 * "MOSS Transcribe Diarize 0.9B" (soniqo, Russian guide), section
   "Implementation notes": the decoder uses symmetric linear INT8 quantisation
   with block 32.
+* "MOSS Transcribe Diarize 0.9B" (soniqo, English guide), section "INT5 vs
+  INT8": the decoder is also deployed with 5-bit weights (the pages give no
+  5-bit layout; the one below is this library's).
 
 Readings where the pages are silent (each listed in the design notes):
 
@@ -26,7 +29,11 @@ Readings where the pages are silent (each listed in the design notes):
   an all-zero (or underflowed, s == 0) block gets q = 0 everywhere;
 * packing: int4 byte j of a row holds element 2j in bits 0-3 and element
   2j+1 in bits 4-7, 4-bit two's complement; int8 is one two's-complement byte
-  per element; scales are binary16 bit patterns in a separate [N, K/32] array;
+  per element; int5 (codes -16..15, 5-bit two's complement) stores a row as
+  K/2 bytes holding the low four bits of every code laid out as int4, then
+  one little-endian 32-bit word per block holding bit 4 of every code of the
+  block, element e of the block at bit e//8 + 4*(e%4) + 16*((e%8)//4);
+  scales are binary16 bit patterns in a separate [N, K/32] array;
 * W is [N, K] (out, in) and Y = X . W^T, exactly, in float64.
 
 Nothing here is blocked, fused or reordered: each function is one step of the
@@ -43,10 +50,20 @@ BLOCK = 32
 
 
 def qrange(bits: int) -> tuple[int, int]:
-    """(qmin, qmax) of symmetric signed ``bits``-bit codes: (-8, 7) or (-128, 127)."""
-    if bits not in (4, 8):
-        raise ValueError(f"bits must be 4 or 8, got {bits}")
+    """(qmin, qmax) of symmetric signed ``bits``-bit codes: (-8, 7), (-16, 15) or (-128, 127)."""
+    if bits not in (4, 5, 8):
+        raise ValueError(f"bits must be 4, 5 or 8, got {bits}")
     return -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+
+
+def int5_high_bit_position(e: int) -> int:
+    """Bit of a block's 32-bit high-bit word that holds bit 4 of the block's element e."""
+    return e // 8 + 4 * (e % 4) + 16 * ((e % 8) // 4)
+
+
+def row_bytes(K: int, bits: int) -> int:
+    """Bytes of one packed row of K codes."""
+    return K * bits // 8
 
 
 def fp16_round(v: np.ndarray) -> np.ndarray:
@@ -109,6 +126,14 @@ def pack(q: np.ndarray, bits: int) -> np.ndarray:
     N, K = q.shape
     if bits == 8:
         return q.astype(np.int8).view(np.uint8).reshape(N, K).copy()
+    if bits == 5:
+        u = q.astype(np.int64) & 0x1F                       # 5-bit two's complement
+        nibbles = pack(((u & 0xF) ^ 8) - 8, 4)              # low four bits, laid out as int4
+        high = np.zeros((N, K // BLOCK), dtype=np.uint32)
+        for e in range(BLOCK):                              # bit 4 of element e of each block
+            bit4 = ((u[:, e::BLOCK] >> 4) & 1).astype(np.uint32)
+            high |= bit4 << np.uint32(int5_high_bit_position(e))
+        return np.concatenate([nibbles, high.astype("<u4").view(np.uint8)], axis=1)
     u = (q.astype(np.int64) & 0xF).astype(np.uint8)        # 4-bit two's complement
     lo = u[:, 0::2]                                         # element 2j -> bits 0-3
     hi = u[:, 1::2]                                         # element 2j+1 -> bits 4-7
@@ -121,6 +146,14 @@ def unpack(packed: np.ndarray, bits: int, K: int) -> np.ndarray:
     N = packed.shape[0]
     if bits == 8:
         return packed.view(np.int8).astype(np.int32).reshape(N, K)
+    if bits == 5:
+        low = unpack(packed[:, :K // 2], 4, K) & 0xF                 # low four bits
+        high = np.ascontiguousarray(packed[:, K // 2:]).view("<u4").astype(np.int64)
+        u = np.empty((N, K), dtype=np.int64)
+        for e in range(BLOCK):
+            bit4 = (high >> int5_high_bit_position(e)) & 1
+            u[:, e::BLOCK] = low[:, e::BLOCK] | (bit4 << 4)
+        return np.where(u >= 16, u - 32, u).astype(np.int32)
     lo = (packed & 0xF).astype(np.int32)
     hi = (packed >> 4).astype(np.int32)
     lo = np.where(lo >= 8, lo - 16, lo)

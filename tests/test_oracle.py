@@ -133,7 +133,7 @@ def _brute_codes(w_row, s_value, bits):
     return out
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 5, 8])
 def test_quantiser_matches_brute_force(bits):
     rng = np.random.default_rng(100 + bits)
     W = (rng.standard_normal((3, 96)) * 0.02).astype(np.float32)
@@ -162,7 +162,8 @@ def test_ties_round_half_even_golden():
     assert y[0, 0] == float(g["y_ones"][0])
 
 
-@pytest.mark.parametrize("bits,name", [(4, "roundtrip_int4.txt"), (8, "roundtrip_int8.txt")])
+@pytest.mark.parametrize("bits,name", [(4, "roundtrip_int4.txt"), (5, "roundtrip_int5.txt"),
+                                       (8, "roundtrip_int8.txt")])
 def test_integer_round_trip_golden(bits, name):
     g = read_kv(name)
     w = np.array([float(v) for v in g["w"]], dtype=np.float32)[None, :]
@@ -201,11 +202,34 @@ def test_pack_unpack_is_a_bijection_on_all_bytes(bits):
     np.testing.assert_array_equal(oracle.pack(q, bits), allb)
 
 
+def test_int5_pack_unpack_is_a_bijection_on_all_bytes():
+    """Every bit of a 20-byte int5 block belongs to exactly one code: any bytes unpack to codes
+    that pack back to the same bytes, and every code -16..15 occurs."""
+    rng = np.random.default_rng(5)
+    b = rng.integers(0, 256, (64, 40)).astype(np.uint8)   # 64 rows of two blocks
+    q = oracle.unpack(b, 5, 64)
+    assert q.min() == -16 and q.max() == 15
+    np.testing.assert_array_equal(oracle.pack(q, 5), b)
+
+
+@pytest.mark.parametrize("e,bit", [(0, 0), (1, 4), (2, 8), (3, 12), (4, 16), (7, 28), (8, 1),
+                                   (12, 17), (29, 23), (31, 31)])
+def test_int5_high_bit_positions(e, bit):
+    """A block whose only nonzero code is -16 (low bits 0000, bit 4 set) at element e: the
+    nibble plane is zero and the high-bit word has exactly the hand-derived bit set."""
+    q = np.zeros((1, 32), dtype=np.int32)
+    q[0, e] = -16
+    p = oracle.pack(q, 5)
+    assert not p[0, :16].any()
+    word = int.from_bytes(bytes(p[0, 16:20]), "little")
+    assert word == 1 << bit
+
+
 # ---------------------------------------------------------------------------
 # special matrices, invariants, linearity, error bound
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 5, 8])
 def test_zero_matrix(bits):
     W = np.zeros((5, 64), dtype=np.float32)
     q, sb = oracle.quantise(W, bits)
@@ -215,7 +239,8 @@ def test_zero_matrix(bits):
     assert not oracle.qgemv_ref(x, oracle.pack(q, bits), sb, bits).any()
 
 
-@pytest.mark.parametrize("bits,diag,sbits", [(4, 1 - 2.0 ** -12, 0x3092), (8, 1 - 2.0 ** -14, 0x2008)])
+@pytest.mark.parametrize("bits,diag,sbits", [(4, 1 - 2.0 ** -12, 0x3092), (5, 1 - 2.0 ** -12, 0x2C44),
+                                             (8, 1 - 2.0 ** -14, 0x2008)])
 def test_identity(bits, diag, sbits):
     K = 64
     W = np.eye(K, dtype=np.float32)
@@ -228,7 +253,7 @@ def test_identity(bits, diag, sbits):
     np.testing.assert_array_equal(y, x.astype(np.float64) * diag)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 5, 8])
 def test_invariants(bits):
     rng = np.random.default_rng(7 + bits)
     W = (rng.standard_normal((16, 256)) * 0.02).astype(np.float32)
@@ -246,7 +271,7 @@ def test_invariants(bits):
     assert np.all((np.sign(q) == np.sign(W)) | (q == 0))
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 5, 8])
 def test_error_bound_against_unquantised_matmul(bits):
     rng = np.random.default_rng(21 + bits)
     W = (rng.standard_normal((24, 128)) * 0.02).astype(np.float32)
@@ -298,7 +323,7 @@ def test_input_errors():
         W[1, 3] = np.inf
         oracle.quantise(W, 8)
     with pytest.raises(ValueError):
-        oracle.qrange(5)
+        oracle.qrange(6)
     with pytest.raises(TypeError):
         oracle.quantise(np.zeros((2, 32), dtype=np.float64), 4)
 
