@@ -843,6 +843,30 @@ def run_batched_decode(layers, groups, device, m: int, peaks, peak_kind, stream,
     return out
 
 
+def run_decode_int5(device, peaks, peak_kind, stream, world, flush, steps=280):
+    """The headline decode step (4 qgemv calls per block, 28 blocks cycled) with int5 weights:
+    0.6875 bytes per weight against int4's 0.5625."""
+    import weight_only_bit_qgemv_b200 as woq
+
+    layers = build_decoder(5, device, FUSED_GROUPS)
+    xs = [workloads.activations(1, group_shape(mem)[1], seed=group_x_seed(mem)).to(device)
+          for _, mem in FUSED_GROUPS]
+    ys = [torch.empty(1, group_shape(mem)[0], device=device) for _, mem in FUSED_GROUPS]
+
+    def step(i):
+        for g, w in enumerate(layers[i]):
+            woq.qgemv(xs[g], w, out=ys[g])
+
+    ms, per_step = time_graph_steps(step, len(layers), steps, 28, stream, world, flush)
+    step_bytes = decode_step_bytes(layers[0])
+    gbs = step_bytes * steps / (ms / 1e3) / 1e9
+    return {"workload": "decoder_block_m1_int5", "dtype": "f32", "bits": 5,
+            "weight_bytes_per_step": step_bytes, "us_per_step": round(ms * 1e3 / steps, 3),
+            "gbs": round(gbs, 1), "launches_per_step": per_step,
+            "timing": f"{steps} steps from CUDA graphs after an L2 flush, 28 blocks cycled",
+            "roofline": roofline(gbs, peaks["hbm_gbs"], "GB/s", "hbm", peak_kind)}
+
+
 def run_fused_epilogues(layers, groups, device, stream, world, flush):
     """The decode-step projections whose neighbours fuse: gate|up with the SwiGLU
     (qgemv_swiglu, the gate|up outputs never written) and down with the residual add
@@ -1136,6 +1160,7 @@ def main(argv=None):
     if not args.no_lm_head:
         configs["lm_head_m1_int8"] = run_lm_head(device, peaks, peak_kind, 8)
         configs["lm_head_m1_int4"] = run_lm_head(device, peaks, peak_kind, 4)
+        configs["lm_head_m1_int5"] = run_lm_head(device, peaks, peak_kind, 5)
         n, k = workloads.LM_HEAD
         lm8 = woq.pack(workloads.weight(n, k, seed=workloads.LM_HEAD_SEED), 8, device)
     if not args.no_prefill:
@@ -1147,6 +1172,8 @@ def main(argv=None):
         if not args.no_prefill:
             configs["prefill_m4096_plus_lm_head"] = run_prefill(
                 layers, groups, device, 4096, peaks, peak_kind, stream, world, flush, lm_head=lm8)
+    if args.m == 1 and not args.unfused:
+        configs["decoder_block_m1_int5"] = run_decode_int5(device, peaks, peak_kind, stream, world, flush)
     if not args.no_fused_epilogues:
         fe = run_fused_epilogues(layers, groups, device, stream, world, flush)
         if fe is not None:

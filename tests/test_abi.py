@@ -46,7 +46,8 @@ def test_argument_checks_return_before_touching_a_device():
     L = _lib.lib()
     ok_ptr = 1 << 20  # never dereferenced: every call below fails validation first
     cases = [
-        (_w(bits=5), _lib.WOQ_EINVAL),
+        (_w(bits=6), _lib.WOQ_EINVAL),
+        (_w(bits=5, k=96), _lib.WOQ_ESHAPE),   # int5 rows must hold whole 128-code groups
         (_w(block=16), _lib.WOQ_EINVAL),
         (_w(k=48), _lib.WOQ_ESHAPE),
         (_w(n=0), _lib.WOQ_ESHAPE),

@@ -11,7 +11,7 @@ from weight_only_bit_qgemv_b200 import container, workloads
 def _weights():
     out = {}
     for name, (n, k, bits) in {"layers.0.qkv": (96, 64, 4), "layers.0.down": (40, 160, 8),
-                               "lm_head": (7, 32, 8)}.items():
+                               "layers.0.o5": (33, 256, 5), "lm_head": (7, 32, 8)}.items():
         p, s = woq.qpack(workloads.weight(n, k, seed=n + k), bits)
         out[name] = woq.PackedWeight(p, s, bits, n, k)
     return out

@@ -25,7 +25,7 @@ def test_random_matches_oracle_bit_exactly(bits, shape):
     np.testing.assert_array_equal(p, p_ref)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [4, 5, 8])
 def test_adversarial_blocks_match_oracle(bits):
     rng = np.random.default_rng(bits)
     W = np.zeros((8, 256), dtype=np.float32)
@@ -51,7 +51,7 @@ def test_golden_fixtures_through_the_c_abi():
     p, s = woq.qpack(torch.from_numpy(w), 4)
     assert list(p.numpy()[0]) == [int(b, 16) for b in g["bytes"]]
     assert int(s.numpy().view(np.uint16)[0, 0]) == int(g["scale"][0], 16)
-    for bits, name in ((4, "roundtrip_int4.txt"), (8, "roundtrip_int8.txt")):
+    for bits, name in ((4, "roundtrip_int4.txt"), (5, "roundtrip_int5.txt"), (8, "roundtrip_int8.txt")):
         g = read_kv(name)
         w = np.array([[float(v) for v in g["w"]]], dtype=np.float32)
         p, s = woq.qpack(torch.from_numpy(w), bits)
@@ -91,7 +91,7 @@ def test_errors():
 
 def test_multithreaded_pack_matches_oracle_on_a_decoder_shape():
     W = workloads.weight(3072, 1024, seed=workloads.layer_seed(0, 4)).numpy()
-    for bits in (4, 8):
+    for bits in (4, 5, 8):
         p, s, p_ref, s_ref = _both(W, bits)
         np.testing.assert_array_equal(s, s_ref)
         np.testing.assert_array_equal(p, p_ref)

@@ -98,13 +98,14 @@ class PackedWeight:
 
 
 def qpack(W: torch.Tensor, bits: int) -> tuple[torch.Tensor, torch.Tensor]:
-    """Host quantiser (C ABI ``qpack``): W float32 [n, k] on the CPU -> (packed, scales)."""
+    """Host quantiser (C ABI ``qpack``): W float32 [n, k] on the CPU -> (packed, scales);
+    bits 4, 5 or 8 (layouts in include/woq.h)."""
     if W.device.type != "cpu" or W.dtype != torch.float32 or W.dim() != 2:
         raise ValueError("qpack takes a 2-D float32 CPU tensor")
     W = W.contiguous()
     n, k = W.shape
-    if bits not in (4, 8) or k % 32:
-        raise ValueError("bits must be 4 or 8 and k a multiple of 32")
+    if bits not in (4, 5, 8) or k % 32:
+        raise ValueError("bits must be 4, 5 or 8 and k a multiple of 32")
     packed = torch.empty(n, k * bits // 8, dtype=torch.uint8)
     scales = torch.empty(n, k // 32, dtype=torch.int16)
     _lib.check(_lib.lib().qpack(_ptr(W), n, k, bits, _ptr(packed), _ptr(scales)), "qpack")

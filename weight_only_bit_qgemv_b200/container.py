@@ -18,7 +18,7 @@ Layout (all integers little-endian):
     32  32  zero
   table, T entries of 128 bytes
     0   64  name, UTF-8, zero-padded (at most 63 bytes)
-    64  4   u32 bits (4 or 8)
+    64  4   u32 bits (4, 5 or 8)
     68  4   u32 block (32)
     72  8   u64 n (rows, out features)
     80  8   u64 k (columns, in features)
@@ -77,8 +77,8 @@ def save(path: str, weights: dict) -> None:
     entries, blobs = [], []
     for name in names:
         w = weights[name]
-        if w.bits not in (4, 8):
-            raise ValueError(f"{name}: bits must be 4 or 8")
+        if w.bits not in (4, 5, 8):
+            raise ValueError(f"{name}: bits must be 4, 5 or 8")
         packed, scales = _host_arrays(w)
         if packed.size != w.n * w.k * w.bits // 8 or scales.size != w.n * (w.k // 32):
             raise ValueError(f"{name}: array sizes do not match n = {w.n}, k = {w.k}")
@@ -121,7 +121,7 @@ def read_table(path: str) -> list[dict]:
         e = {"name": name.rstrip(b"\0").decode(), "bits": bits, "block": block, "n": n, "k": k,
              "off_packed": off_p, "off_scales": off_s, "crc_packed": crc_p, "crc_scales": crc_s,
              "bytes_packed": n * k * bits // 8, "bytes_scales": n * (k // 32) * 2}
-        if bits not in (4, 8) or block != 32 or k % 32 or n < 1:
+        if bits not in (4, 5, 8) or block != 32 or k % 32 or n < 1:
             raise ContainerError(f"{e['name']}: bad shape or format")
         if off_p % ALIGN or off_s % ALIGN or off_p < data_off or off_s < data_off:
             raise ContainerError(f"{e['name']}: data not 64-byte aligned or inside the table")

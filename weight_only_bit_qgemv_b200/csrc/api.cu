@@ -23,9 +23,10 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 int check_weight(const woq_weight *w) {
   if (!w || !w->packed || !w->scales) return WOQ_EINVAL;
-  if (w->bits != 4 && w->bits != 8) return WOQ_EINVAL;
+  if (w->bits != 4 && w->bits != 5 && w->bits != 8) return WOQ_EINVAL;
   if (w->block != 32) return WOQ_EINVAL;
   if (w->n <= 0 || w->k <= 0 || w->k % 32 != 0) return WOQ_ESHAPE;
+  if (w->bits == 5 && w->k % 128 != 0) return WOQ_ESHAPE;  // int5 rows on 16-byte boundaries
   if (w->n > INT32_MAX || w->k > INT32_MAX / 8) return WOQ_ESHAPE;
   if (!aligned(w->packed, 64) || !aligned(w->scales, 64)) return WOQ_EALIGN;
   return WOQ_OK;
@@ -89,6 +90,10 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
   rc = woq::current_device(&dev);
   if (rc != WOQ_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (w->bits == 5) {  // int5: the CUDA-core kernel only
+    if (path != WOQ_GEMV_AUTO && path != WOQ_GEMV_CUDA_CORE) return WOQ_EINVAL;
+    return woq::launch_gemv_fp32(x, m, *w, y, s, dev, true);
+  }
   if (path == WOQ_GEMV_INT8_TC) {
     rc = woq::launch_gemv_i8tc(x, m, *w, y, s, dev);
     return rc == 1 ? WOQ_ESHAPE : rc;
@@ -208,9 +213,11 @@ static int plan_sm_count() {
 // kernel below that.
 constexpr int64_t kSplitMinM = 24;
 
-static int resolve_path(int32_t path, int64_t m) {
-  if (path == WOQ_PATH_AUTO)
+static int resolve_path(int32_t path, int64_t m, int32_t bits) {
+  if (path == WOQ_PATH_AUTO) {
+    if (bits == 5) return WOQ_PATH_FP32;  // int5: the CUDA-core kernel only
     return m >= 128 ? WOQ_PATH_BF16_TC : m >= kSplitMinM ? WOQ_PATH_SPLIT_TC : WOQ_PATH_FP32;
+  }
   return path;
 }
 
@@ -222,8 +229,8 @@ static bool known_path(int32_t path) {
 size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path) {
   if (woq::check_weight(w) != WOQ_OK || m < 1) return 0;
   if (!known_path(path)) return 0;
-  const int p = resolve_path(path, m);
-  if (p == WOQ_PATH_FP32) return 0;
+  const int p = resolve_path(path, m, w->bits);
+  if (p == WOQ_PATH_FP32 || w->bits == 5) return 0;
   return woq::plan_gemm_tc(m, w->n, w->k, plan_sm_count(), SIZE_MAX, p == WOQ_PATH_SPLIT_TC).total;
 }
 
@@ -235,7 +242,8 @@ int qgemm(const float *X, int64_t m, const woq_weight *w, float *Y, int32_t path
   if (m < 1 || m > INT32_MAX) return WOQ_EINVAL;
   if (!known_path(path)) return WOQ_EINVAL;
   if (!woq::aligned(X, 16) || !woq::aligned(Y, 16)) return WOQ_EALIGN;
-  const int p = resolve_path(path, m);
+  const int p = resolve_path(path, m, w->bits);
+  if (w->bits == 5 && p != WOQ_PATH_FP32) return WOQ_EINVAL;  // no tensor-core int5 form
   if (p == WOQ_PATH_FP32 && w->k > 32768) return WOQ_ESHAPE;
   woq::GemmPlan plan;
   if (p != WOQ_PATH_FP32) {

@@ -223,3 +223,73 @@ __device__ __forceinline__ void block_int8(const float4 *__restrict__ xs4, int u
 
 }  // namespace gemv
 }  // namespace woq
+
+namespace woq {
+namespace gemv {
+
+// int5: one 32-bit word of low nibbles (elements e0..e7, e_p in bits 4p..4p+3, the int4 layout)
+// and `nb`, the complemented fifth bits of the same elements (bit 4j for e_j, bit 16+4j for
+// e_{4+j}; built by int5_fifth_bits). Each field becomes the offset-binary value
+// u = code + 16 in the low mantissa bits of 2^23 (one LOP3 for the nibble, one for the fifth
+// bit, moved just above its nibble: left by 4 for e_j, right by 12 for e_{4+j}); one exact
+// packed subtraction removes 2^23 + 16, leaving the exact pairs p[j] = (q_j, q_{4+j}) * 2^(4j),
+// as unpack_int4_word gives for int4.
+__device__ __forceinline__ void unpack_int5_word(uint32_t w, uint32_t nb, float2 (&p)[4]) {
+  const uint32_t hi = w >> 16, nb4 = nb << 4, nbh = nb >> 12;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t mask = 0xFu << (4 * j);
+    const uint32_t m5 = 0x10u << (4 * j);
+    const float bias = 8388608.0f + 16.0f * static_cast<float>(1u << (4 * j));
+    const float lo_f = __uint_as_float(((w & mask) | 0x4B000000u) | (nb4 & m5));
+    const float hi_f = __uint_as_float(((hi & mask) | 0x4B000000u) | (nbh & m5));
+    p[j] = __fadd2_rn(make_float2(lo_f, hi_f), make_float2(-bias, -bias));
+  }
+}
+
+// The block's high-bit word H holds bit 4 of element e at bit e/8 + 4(e%4) + 16((e%8)/4); for
+// the block's word i (elements 8i..8i+7) this returns their complemented fifth bits, e_{8i+j}
+// at bit 4j and e_{8i+4+j} at bit 16+4j, as unpack_int5_word expects.
+__device__ __forceinline__ uint32_t int5_fifth_bits(uint32_t H, int i) {
+  return (~(H >> i)) & 0x11111111u;
+}
+
+// int5: one block of R rows (low nibbles `wv`, high-bit words `hw`) against MT x rows; the x
+// units and the 2^(4j) folding are those of chunk_int4.
+template <int MT, int R>
+__device__ __forceinline__ void chunk_int5(const float4 *__restrict__ xs4, int units_row, int c,
+                                           const uint4 (&wv)[R], const uint32_t (&hw)[R],
+                                           const float (&sc)[R], float (&acc)[R][MT]) {
+  float4 xv[MT][8];
+#pragma unroll
+  for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) xv[mm][t] = xs4[mm * units_row + swz(8 * c + t)];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float2 a2[MT][4];
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) a2[mm][j] = make_float2(0.f, 0.f);
+    const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 p[4];
+      unpack_int5_word(ws[i], int5_fifth_bits(hw[r], i), p);
+#pragma unroll
+      for (int mm = 0; mm < MT; ++mm) {
+        const float4 xa = xv[mm][2 * i], xb = xv[mm][2 * i + 1];
+        a2[mm][0] = __ffma2_rn(p[0], make_float2(xa.x, xa.y), a2[mm][0]);
+        a2[mm][1] = __ffma2_rn(p[1], make_float2(xa.z, xa.w), a2[mm][1]);
+        a2[mm][2] = __ffma2_rn(p[2], make_float2(xb.x, xb.y), a2[mm][2]);
+        a2[mm][3] = __ffma2_rn(p[3], make_float2(xb.z, xb.w), a2[mm][3]);
+      }
+    }
+#pragma unroll
+    for (int mm = 0; mm < MT; ++mm) acc[r][mm] = fmaf(sc[r], fold_int4(a2[mm]), acc[r][mm]);
+  }
+}
+
+}  // namespace gemv
+}  // namespace woq

@@ -45,6 +45,35 @@ template <int BITS, int MT, int RW, bool SMEM>
 __device__ __forceinline__ void rows_dot(const float4 *__restrict__ xs4, int units_row, int spr,
                                          int lane, const uint8_t *codes, size_t row_stride,
                                          const uint16_t *scs, int valid, float (&acc)[RW][MT]) {
+  if constexpr (BITS == 5) {
+    // int5: a block's 16 bytes of low nibbles at 16 b, its high-bit word at k/2 + 4 b
+    const int half = spr * 16;
+    for (int b = lane; b < spr; b += 32) {
+      uint4 lo[RW];
+      uint32_t hw[RW];
+      float sc[RW];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const uint8_t *pr = codes + r * row_stride;
+        if (SMEM || r < valid) {
+          if constexpr (SMEM) {
+            lo[r] = *reinterpret_cast<const uint4 *>(pr + b * 16);
+            hw[r] = *reinterpret_cast<const uint32_t *>(pr + half + b * 4);
+            sc[r] = half_bits_to_float(scs[r * spr + b]);
+          } else {
+            lo[r] = ptx::ldg_stream_v4(pr + b * 16);
+            hw[r] = __ldg(reinterpret_cast<const uint32_t *>(pr + half + b * 4));
+            sc[r] = half_bits_to_float(__ldg(scs + r * spr + b));
+          }
+        } else {
+          lo[r] = make_uint4(0u, 0u, 0u, 0u);
+          hw[r] = 0xFFFFFFFFu;  // with zero nibbles: code -16 times a zero scale
+          sc[r] = 0.f;
+        }
+      }
+      chunk_int5<MT, RW>(xs4, units_row, b, lo, hw, sc, acc);
+    }
+  } else {
   constexpr int kBlockBytes = BITS * 4;  // 16 (int4) or 32 (int8)
   for (int b = lane; b < spr; b += 32) {
     uint4 lo[RW], hi[RW];
@@ -72,6 +101,7 @@ __device__ __forceinline__ void rows_dot(const float4 *__restrict__ xs4, int uni
       chunk_int4<MT, RW>(xs4, units_row, b, lo, sc, acc);
     else
       block_int8<MT, RW>(xs4, units_row, b, lo, hi, sc, acc);
+  }
   }
 }
 
@@ -144,7 +174,7 @@ __global__ void __launch_bounds__(kThreads)
       b = src[1];
     }
     float4 pa = a, pb = b;
-    if constexpr (BITS == 4) {
+    if constexpr (BITS != 8) {  // int4 and int5: nibble pairs
       pa = make_float4(a.x, b.x, a.y, b.y);
       pb = make_float4(a.z, b.z, a.w, b.w);
     }
@@ -350,7 +380,7 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
       b = src[1];
     }
     float4 pa = a, pb = b;
-    if constexpr (BITS == 4) {
+    if constexpr (BITS != 8) {  // int4 and int5: nibble pairs
       pa = make_float4(a.x, b.x, a.y, b.y);
       pb = make_float4(a.z, b.z, a.w, b.w);
     }
@@ -664,11 +694,15 @@ int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
     default: rc = try_bulk<BITS, 8>(x, m, w, y, s, dev, pdl); break;
   }
   if (rc != 1) return rc;
-  switch (mt) {
-    case 1: return pick_ru<BITS, 1>(x, m, w, y, s, dev, pdl);
-    case 2: return pick_ru<BITS, 2>(x, m, w, y, s, dev, pdl);
-    case 4: return pick_ru<BITS, 4>(x, m, w, y, s, dev, pdl);
-    default: return pick_ru<BITS, 8>(x, m, w, y, s, dev, pdl);
+  if constexpr (BITS == 5) {
+    return WOQ_ESHAPE;  // int5: the staged kernel only
+  } else {
+    switch (mt) {
+      case 1: return pick_ru<BITS, 1>(x, m, w, y, s, dev, pdl);
+      case 2: return pick_ru<BITS, 2>(x, m, w, y, s, dev, pdl);
+      case 4: return pick_ru<BITS, 4>(x, m, w, y, s, dev, pdl);
+      default: return pick_ru<BITS, 8>(x, m, w, y, s, dev, pdl);
+    }
   }
 }
 
@@ -782,18 +816,23 @@ int read_gemv_timeout_flag(int clear, unsigned *value) {
 
 int launch_gemv_fp32(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                      const DevInfo &dev, bool pdl) {
-  return w.bits == 4 ? pick_mt<4>(x, m, w, y, s, dev, pdl) : pick_mt<8>(x, m, w, y, s, dev, pdl);
+  return w.bits == 4 ? pick_mt<4>(x, m, w, y, s, dev, pdl)
+       : w.bits == 5 ? pick_mt<5>(x, m, w, y, s, dev, pdl)
+                     : pick_mt<8>(x, m, w, y, s, dev, pdl);
 }
 
 int launch_gemv_swiglu(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                        const DevInfo &dev) {
-  const int rc = w.bits == 4 ? swiglu_bulk<4>(x, m, w, y, s, dev) : swiglu_bulk<8>(x, m, w, y, s, dev);
+  const int rc = w.bits == 4 ? swiglu_bulk<4>(x, m, w, y, s, dev)
+               : w.bits == 5 ? swiglu_bulk<5>(x, m, w, y, s, dev)
+                             : swiglu_bulk<8>(x, m, w, y, s, dev);
   return rc == 1 ? WOQ_ESHAPE : rc;
 }
 
 int launch_gemv_residual(const float *x, int64_t m, const woq_weight &w, const float *r, float *y,
                          cudaStream_t s, const DevInfo &dev) {
   const int rc = w.bits == 4 ? residual_bulk<4>(x, m, w, r, y, s, dev)
+               : w.bits == 5 ? residual_bulk<5>(x, m, w, r, y, s, dev)
                              : residual_bulk<8>(x, m, w, r, y, s, dev);
   return rc == 1 ? WOQ_ESHAPE : rc;
 }
@@ -813,7 +852,9 @@ int launch_gemv_argmax(const float *x, int64_t m, const woq_weight &w, int64_t *
   if (cudaLaunchKernelEx(&cfg, argmax_init_kernel, keys, static_cast<int>(m)) != cudaSuccess)
     return WOQ_ECUDA;
   count_launches(1);
-  const int rc = w.bits == 4 ? argmax_bulk<4>(x, m, w, keys, s, dev) : argmax_bulk<8>(x, m, w, keys, s, dev);
+  const int rc = w.bits == 4 ? argmax_bulk<4>(x, m, w, keys, s, dev)
+               : w.bits == 5 ? argmax_bulk<5>(x, m, w, keys, s, dev)
+                             : argmax_bulk<8>(x, m, w, keys, s, dev);
   if (rc == 1) return WOQ_ESHAPE;
   if (rc != WOQ_OK) return rc;
   if (cudaLaunchKernelEx(&cfg, argmax_final_kernel, keys, val, static_cast<int>(m)) != cudaSuccess)

@@ -108,7 +108,7 @@ template <int BITS, int MT>
 __device__ __forceinline__ void stage_dots(const float4 *xs4, int units_row, const uint8_t *codes,
                                            const uint16_t *scs, int nr, int k, int parts, int warp,
                                            int lane, float *psum) {
-  constexpr int kBlockBytes = BITS * 4;  // 16 (int4) or 32 (int8)
+  constexpr int kBlockBytes = BITS == 8 ? 32 : 16;  // int4/int5: a block's (low) nibbles
   const int spr = k >> 5;
   const size_t row_bytes = static_cast<size_t>(k) * BITS / 8;
   for (int job = warp; job < nr * parts; job += kNW) {
@@ -125,10 +125,14 @@ __device__ __forceinline__ void stage_dots(const float4 *xs4, int units_row, con
       lo[0] = *reinterpret_cast<const uint4 *>(crow + b * kBlockBytes);
       if constexpr (BITS == 8) hi[0] = *reinterpret_cast<const uint4 *>(crow + b * kBlockBytes + 16);
       sc[0] = half_bits_to_float(srow[b]);
-      if constexpr (BITS == 4)
+      if constexpr (BITS == 4) {
         chunk_int4<MT, 1>(xs4, units_row, b, lo, sc, acc);
-      else
+      } else if constexpr (BITS == 5) {  // the block's high-bit word follows the row's nibbles
+        const uint32_t hw[1] = {*reinterpret_cast<const uint32_t *>(crow + spr * 16 + b * 4)};
+        chunk_int5<MT, 1>(xs4, units_row, b, lo, hw, sc, acc);
+      } else {
         block_int8<MT, 1>(xs4, units_row, b, lo, hi, sc, acc);
+      }
     }
 #pragma unroll
     for (int mm = 0; mm < MT; ++mm) {
@@ -240,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1)
         b = __ldcg(src + 1);
       }
       float4 pa = a, pb = b;
-      if (it.bits == 4) {  // int4 pairs (q_j, q_{4+j}) meet (x_j, x_{4+j})
+      if (it.bits != 8) {  // int4/int5 pairs (q_j, q_{4+j}) meet (x_j, x_{4+j})
         pa = make_float4(a.x, b.x, a.y, b.y);
         pb = make_float4(a.z, b.z, a.w, b.w);
       }
@@ -270,6 +274,8 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1)
       const uint16_t *scs = reinterpret_cast<const uint16_t *>(stage + nr * rbytes);
       if (it.bits == 4)
         stage_dots<4, MT>(xs4, units_row, stage, scs, nr, k, it.parts, warp, lane, psum);
+      else if (it.bits == 5)
+        stage_dots<5, MT>(xs4, units_row, stage, scs, nr, k, it.parts, warp, lane, psum);
       else
         stage_dots<8, MT>(xs4, units_row, stage, scs, nr, k, it.parts, warp, lane, psum);
       asm volatile("bar.sync 1, %0;" ::"n"(kNW * 32) : "memory");

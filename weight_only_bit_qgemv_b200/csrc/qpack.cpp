@@ -1,8 +1,10 @@
 // Host-side quantiser: float32 W [n, k] -> packed int4/int8 codes + binary16 block scales.
 //
 // Formats: int4 in blocks of 32 ("MOSS-Transcribe-Diarize -- LiteRT (TFLite)", section
-// "Files": the q4b32 production decoder) and symmetric linear INT8 in blocks of 32 (soniqo
-// Russian guide, section "Implementation notes"). Rule per row r and block j:
+// "Files": the q4b32 production decoder), symmetric linear INT8 in blocks of 32 (soniqo
+// Russian guide, section "Implementation notes") and 5-bit codes in blocks of 32 (soniqo
+// English guide, section "INT5 vs INT8", which gives no layout: the one written here is this
+// library's, documented in include/woq.h). Rule per row r and block j:
 //   a = max |w| over the block (exact)
 //   s = binary16(round-half-even((double)a / qmax))
 //   q = clamp(round-half-even((double)w / (double)s), qmin, qmax), or 0 when s == 0.
@@ -82,6 +84,16 @@ int pack_rows(const float *W, int64_t r0, int64_t r1, int64_t k, int bits, uint8
       }
       if (bits == 8) {
         for (int i = 0; i < 32; ++i) pr[j * 32 + i] = static_cast<uint8_t>(static_cast<int8_t>(q[i]));
+      } else if (bits == 5) {
+        // low four bits as int4 in the row's first k/2 bytes; bit 4 of element i of the block in
+        // bit (i / 8 + 4 * (i % 4) + 16 * ((i % 8) / 4)) of the block's word after them
+        uint32_t high = 0;
+        for (int i = 0; i < 16; ++i)
+          pr[j * 16 + i] = static_cast<uint8_t>((q[2 * i] & 0xF) | ((q[2 * i + 1] & 0xF) << 4));
+        for (int i = 0; i < 32; ++i)
+          high |= static_cast<uint32_t>((q[i] >> 4) & 1) << (i / 8 + 4 * (i % 4) + 16 * ((i % 8) / 4));
+        uint8_t *ph = pr + k / 2 + j * 4;
+        for (int b = 0; b < 4; ++b) ph[b] = static_cast<uint8_t>(high >> (8 * b));
       } else {
         for (int i = 0; i < 16; ++i)
           pr[j * 16 + i] = static_cast<uint8_t>((q[2 * i] & 0xF) | ((q[2 * i + 1] & 0xF) << 4));
@@ -96,7 +108,7 @@ int pack_rows(const float *W, int64_t r0, int64_t r1, int64_t k, int bits, uint8
 extern "C" int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed,
                      uint16_t *scales) {
   if (!W || !packed || !scales) return WOQ_EINVAL;
-  if (bits != 4 && bits != 8) return WOQ_EINVAL;
+  if (bits != 4 && bits != 5 && bits != 8) return WOQ_EINVAL;
   if (n <= 0 || k <= 0 || k % 32 != 0) return WOQ_ESHAPE;
   if (std::fegetround() != FE_TONEAREST) return WOQ_EINVAL;  // nearbyint must round to even
 
