@@ -1118,10 +1118,24 @@ def main(argv=None):
     ap.add_argument("--no-lm-head", action="store_true")
     ap.add_argument("--no-fused-epilogues", action="store_true")
     ap.add_argument("--no-batched", action="store_true", help="skip the M=64 / M=4096 legs")
+    ap.add_argument("--legs", default="all",
+                    help="comma list of legs to run (the headline decode always runs): chain, int5, "
+                         "single, lm_head, prefill, batched, epilogues, cpu; default all")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    legs = {"chain", "int5", "single", "lm_head", "prefill", "batched", "epilogues", "cpu"}
+    if args.legs != "all":
+        want = {x.strip() for x in args.legs.split(",") if x.strip()}
+        if not want <= legs | {"decode"}:
+            ap.error(f"--legs takes {sorted(legs)}")
+        legs = want
+    args.no_prefill = args.no_prefill or "prefill" not in legs
+    args.no_lm_head = args.no_lm_head or "lm_head" not in legs
+    args.no_batched = args.no_batched or "batched" not in legs
+    args.no_fused_epilogues = args.no_fused_epilogues or "epilogues" not in legs
+    args.no_cpu_baseline = args.no_cpu_baseline or "cpu" not in legs
     world, rank, local = dist_setup()
     if args.impl == "reference":
         out = run_reference(args, world, rank)
@@ -1138,11 +1152,16 @@ def main(argv=None):
     device = torch.device("cuda", local)
     flush = L2Flush(device)
     stream = torch.cuda.Stream(device)
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push("decode")
     out, layers, groups, xs = run_decode(args, world, local, peaks, peak_kind, flush)
+    nvtx.range_pop()
     configs = {}
     chain_step = None
-    if not args.unfused and args.m <= 8:
+    if not args.unfused and args.m <= 8 and "chain" in legs:
+        nvtx.range_push("chain")
         ch, clayers, chain_step = run_decode_chain(args, world, local, peaks, peak_kind, flush, layers)
+        nvtx.range_pop()
         calls = {k: out[k] for k in ("value", "ms_per_step", "config", "hbm_frac", "clocks", "e2e",
                                      "gpu_launches", "roofline", "per_kernel")}
         if args.decode_step == "chain" or (args.decode_step == "best" and ch["value"] > out["value"]):
@@ -1155,32 +1174,47 @@ def main(argv=None):
     configs["decoder_block_m1"] = {"workload": out["config"]["workload"], "dtype": "f32",
                                    "gbs": out["value"], "us_per_step": round(out["ms_per_step"] * 1e3, 3),
                                    "roofline": out["roofline"], "note": "the headline line itself"}
-    configs["single_qgemv_m1"] = run_single_qgemv(device, peaks, peak_kind, stream, world, flush)
+    if "single" in legs:
+        nvtx.range_push("single_qgemv_m1")
+        configs["single_qgemv_m1"] = run_single_qgemv(device, peaks, peak_kind, stream, world, flush)
+        nvtx.range_pop()
     lm8 = None
     if not args.no_lm_head:
-        configs["lm_head_m1_int8"] = run_lm_head(device, peaks, peak_kind, 8)
-        configs["lm_head_m1_int4"] = run_lm_head(device, peaks, peak_kind, 4)
-        configs["lm_head_m1_int5"] = run_lm_head(device, peaks, peak_kind, 5)
+        for bits in (8, 4, 5):
+            nvtx.range_push(f"lm_head_m1_int{bits}")
+            configs[f"lm_head_m1_int{bits}"] = run_lm_head(device, peaks, peak_kind, bits)
+            nvtx.range_pop()
+    if not args.no_batched:
         n, k = workloads.LM_HEAD
         lm8 = woq.pack(workloads.weight(n, k, seed=workloads.LM_HEAD_SEED), 8, device)
     if not args.no_prefill:
+        nvtx.range_push("prefill_m512")
         configs["prefill_m512"] = run_prefill(layers, groups, device, 512, peaks, peak_kind,
                                               stream, world, flush)
+        nvtx.range_pop()
     if not args.no_batched:
+        nvtx.range_push("decoder_m64_plus_lm_head")
         configs["decoder_m64_plus_lm_head"] = run_batched_decode(
             layers, groups, device, 64, peaks, peak_kind, stream, world, flush, lm_head=lm8)
+        nvtx.range_pop()
         if not args.no_prefill:
+            nvtx.range_push("prefill_m4096_plus_lm_head")
             configs["prefill_m4096_plus_lm_head"] = run_prefill(
                 layers, groups, device, 4096, peaks, peak_kind, stream, world, flush, lm_head=lm8)
-    if args.m == 1 and not args.unfused:
+            nvtx.range_pop()
+    if args.m == 1 and not args.unfused and "int5" in legs:
+        nvtx.range_push("decoder_block_m1_int5")
         configs["decoder_block_m1_int5"] = run_decode_int5(device, peaks, peak_kind, stream, world, flush)
+        nvtx.range_pop()
     if not args.no_fused_epilogues:
+        nvtx.range_push("fused_epilogues")
         fe = run_fused_epilogues(layers, groups, device, stream, world, flush)
+        nvtx.range_pop()
         if fe is not None:
             out["fused_epilogues"] = fe
     if rank == 0 and not args.no_cpu_baseline and args.m == 1 and not args.unfused:
-        legs, parity = cpu_legs(groups, layers[0], xs)
-        out["cpu_baseline"] = legs.pop("decoder_block_m1")
+        cpu, parity = cpu_legs(groups, layers[0], xs)
+        out["cpu_baseline"] = cpu.pop("decoder_block_m1")
         out["parity"] = parity
         if chain_step is not None:
             out["parity_chain"] = chain_parity(chain_step, oracle_chain_block0())
@@ -1190,7 +1224,7 @@ def main(argv=None):
                   "prefill_m4096": "prefill_m4096_plus_lm_head"}
         for leg, cfg in key_of.items():
             if cfg in configs:
-                configs[cfg]["cpu_baseline"] = legs[leg]
+                configs[cfg]["cpu_baseline"] = cpu[leg]
     out["configs"] = configs
     if rank == 0:
         print(json.dumps(out), flush=True)

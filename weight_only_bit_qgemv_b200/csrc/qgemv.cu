@@ -588,6 +588,9 @@ int pick_ru(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
 
 // Bulk-pipeline launch. Returns 1 (not launched) when the shape does not suit it.
 constexpr size_t kStageTarget = 20 * 1024;   // bytes per ring stage to aim for
+// 8-warp (bandwidth-bound, wide-matrix) launches: a larger stage lets a warp take more rows
+// (more independent work per lane between waits); two such stages still fit the budget.
+constexpr size_t kStageTargetWide = 36 * 1024;
 constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
 
 template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
@@ -631,10 +634,15 @@ int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cuda
   return WOQ_OK;
 }
 
-// Rows per warp for NW compute warps: as many as fit a stage of about kStageTarget bytes.
-inline int bulk_rows_per_warp(int nw, int rw_max, size_t row_total) {
+// Rows per warp for NW compute warps: as many as fit a stage of about kStageTarget bytes; for
+// 8 warps over a wide matrix, more (up to kStageTargetWide) while the tiles still number at
+// least two per SM.
+inline int bulk_rows_per_warp(int nw, int rw_max, size_t row_total, int64_t n = 0, int sms = 0) {
   int rw = rw_max;
   while (rw > 1 && static_cast<size_t>(nw) * rw * row_total > kStageTarget) rw /= 2;
+  while (nw == 8 && rw < rw_max && static_cast<size_t>(nw) * rw * 2 * row_total <= kStageTargetWide &&
+         n / (nw * rw * 2) >= 2 * static_cast<int64_t>(sms))
+    rw *= 2;
   return rw;
 }
 
@@ -643,7 +651,7 @@ int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cud
                    const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes,
                    unsigned long long *keys = nullptr, const float *resid = nullptr) {
   // More rows per warp only where registers allow.
-  int rw = bulk_rows_per_warp(NW, NW == 16 ? 2 : MT <= 2 ? 4 : 2, row_total);
+  int rw = bulk_rows_per_warp(NW, NW == 16 ? 2 : MT <= 2 ? 4 : 2, row_total, w.n, dev.sm_count);
   const size_t stage_bytes = (static_cast<size_t>(NW) * rw * row_total + 127) & ~size_t(127);
   if (kBulkHeader + x_bytes + stage_bytes > kCtaSmemBudget) return 1;
   if (w.n < NW * rw) rw = 1;  // tiny n: one row per warp, all from global memory
