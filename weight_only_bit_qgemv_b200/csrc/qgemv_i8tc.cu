@@ -63,7 +63,7 @@ constexpr int kMaxA = 10;     // s8 code tiles
 constexpr int kMaxRaw = 12;   // packed int4 tiles
 constexpr int kMaxSlots = 16; // tensor-memory stage slots
 constexpr int kMaxM = 4;
-constexpr int kScaleChunk = 8;  // stages of scales fetched ahead by each read-out lane
+constexpr int kScaleChunk = 4;  // stages of scales fetched ahead by each read-out lane
 constexpr long long kWaitLimit = 1LL << 32;   // cycles (~2 s)
 constexpr long long kDrainLimit = 1LL << 31;  // cycles (~1 s)
 
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // (4) read-out: TMEM lane = weight row; per stage slot nb columns. The CTA's stages are
     // walked as one sequence over its units; each row's binary16 scales (8 bytes a stage) are
-    // loaded a chunk of eight stages ahead, the first chunk before the wait on the preceding
+    // loaded a chunk of four stages ahead, the first chunk before the wait on the preceding
     // grid, so no stage waits on a scale load.
     int slot = 0;
     uint32_t sph = 0;
@@ -408,41 +408,47 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         ptx::tc_fence_after();
         const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(slot * 4 * nb);
-        // block j's columns start at j * nb: 3 m of them hold its sums (column 3 a + i)
+        // block j's columns start at j * nb: 3 m of them hold its sums (column 3 a + i); the
+        // blocks are read in groups of G (all four at once for m <= 2, pairs above, so that
+        // the loaded columns fit in registers)
         constexpr int C = M == 1 ? 4 : M == 2 ? 8 : 16;
-        uint32_t r[kBlocksPerStage][C];
+        constexpr int G = M <= 2 ? kBlocksPerStage : 2;
+        const __half2 h01 = *reinterpret_cast<const __half2 *>(&scur[i].x);
+        const __half2 h23 = *reinterpret_cast<const __half2 *>(&scur[i].y);
+        const float sc[kBlocksPerStage] = {__low2float(h01), __high2float(h01), __low2float(h23),
+                                           __high2float(h23)};
 #pragma unroll
-        for (int j = 0; j < kBlocksPerStage; ++j) {
-          if constexpr (C == 4) ptx::tmem_ld_32x32b_x4(tb + j * nb, r[j]);
-          else if constexpr (C == 8) ptx::tmem_ld_32x32b_x8(tb + j * nb, r[j]);
-          else ptx::tmem_ld_32x32b_x16(tb + j * nb, r[j]);
+        for (int j0 = 0; j0 < kBlocksPerStage; j0 += G) {
+          uint32_t r[G][C];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            if constexpr (C == 4) ptx::tmem_ld_32x32b_x4(tb + (j0 + g) * nb, r[g]);
+            else if constexpr (C == 8) ptx::tmem_ld_32x32b_x8(tb + (j0 + g) * nb, r[g]);
+            else ptx::tmem_ld_32x32b_x16(tb + (j0 + g) * nb, r[g]);
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) ptx::tmem_ld_wait(r[g]);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const int b = st * kBlocksPerStage + j0 + g;
+            if (b < spr) {
+#pragma unroll
+              for (int a = 0; a < M; ++a) {
+                const int c = a * 3;
+                const float t = fmaf(static_cast<float>(static_cast<int>(r[g][c + 2])), 6.103515625e-05f,
+                                     fmaf(static_cast<float>(static_cast<int>(r[g][c + 1])), 0.0078125f,
+                                          static_cast<float>(static_cast<int>(r[g][c]))));
+                acc[a] = fmaf(sc[j0 + g] * cexp[a * nblk + (b - blk0)], t, acc[a]);
+              }
+            }
+          }
         }
-#pragma unroll
-        for (int j = 0; j < kBlocksPerStage; ++j) ptx::tmem_ld_wait(r[j]);
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.accempty[slot]);
         if (++slot == slots) {
           slot = 0;
           sph ^= 1;
-        }
-        const __half2 h01 = *reinterpret_cast<const __half2 *>(&scur[i].x);
-        const __half2 h23 = *reinterpret_cast<const __half2 *>(&scur[i].y);
-        const float sc[kBlocksPerStage] = {__low2float(h01), __high2float(h01), __low2float(h23),
-                                           __high2float(h23)};
-#pragma unroll
-        for (int j = 0; j < kBlocksPerStage; ++j) {
-          const int b = st * kBlocksPerStage + j;
-          if (b < spr) {
-#pragma unroll
-            for (int a = 0; a < M; ++a) {
-              const int c = a * 3;
-              const float t = fmaf(static_cast<float>(static_cast<int>(r[j][c + 2])), 6.103515625e-05f,
-                                   fmaf(static_cast<float>(static_cast<int>(r[j][c + 1])), 0.0078125f,
-                                        static_cast<float>(static_cast<int>(r[j][c]))));
-              acc[a] = fmaf(sc[j] * cexp[a * nblk + (b - blk0)], t, acc[a]);
-            }
-          }
         }
         if (st == s1 - 1) {  // the unit's last stage: its outputs are complete
           if (splits == 1) {
