@@ -14,6 +14,8 @@
  *     int4 in blocks of 32 ("q4b32").
  *   - "MOSS Transcribe Diarize 0.9B" (soniqo, Russian guide), "Implementation notes":
  *     symmetric linear INT8 quantisation with block 32 for the decoder.
+ *   - "MOSS Transcribe Diarize 0.9B" (soniqo, English guide), "INT5 vs INT8": names a 5-bit
+ *     width beside INT8 but no format; the int5 layout below is this library's own.
  *
  * Packed layout (fixed; qpack produces it bit-exactly):
  *   bits == 4: row r of W occupies k/2 bytes at packed + r*k/2. Byte j holds element 2j in
@@ -21,9 +23,15 @@
  *              in [-8, 7].
  *   bits == 8: row r occupies k bytes at packed + r*k, one two's-complement byte per
  *              element, codes in [-128, 127].
+ *   bits == 5: (k % 128 == 0) row r occupies 5k/8 bytes at packed + r*5k/8, codes in
+ *              [-16, 15], scale max|w|/15. The first k/2 bytes hold each code's low four
+ *              bits laid out as bits == 4 does; then k/32 little-endian 32-bit words, word b
+ *              holding bit 4 of block b's codes: element e (0..31) of the block at bit
+ *              e/8 + 4*(e%4) + 16*((e%8)/4), so that one shift and mask per 8 codes lines
+ *              the fifth bits up with the low nibbles of a 32-bit load.
  *   scales:    binary16 bit patterns, [n, k/32] row-major; element (r, j) scales codes
  *              k in [32j, 32j+32) of row r. W_hat[r, c] = scale[r, c/32] * code[r, c].
- *   All codes a container may hold are decoded, including -8 / -128, which qpack never
+ *   All codes a container may hold are decoded, including -8 / -16 / -128, which qpack never
  *   emits.
  *
  * Conventions for every call:
@@ -47,7 +55,8 @@ extern "C" {
 
 /* Status codes. */
 #define WOQ_OK          0
-#define WOQ_EINVAL     -1  /* null pointer, bits not 4/8, block not 32, m out of range, bad path */
+#define WOQ_EINVAL     -1  /* null pointer, bits not 4/5/8, block not 32, m out of range,    */
+                           /* bad path, or a path that does not take int5                 */
 #define WOQ_ESHAPE     -2  /* n or k <= 0, k % 32 != 0, or a size above a documented limit    */
 #define WOQ_EALIGN     -3  /* packed/scales not 64-byte aligned, or x/y not 16-byte aligned    */
 #define WOQ_ERANGE     -4  /* qpack: non-finite weight, or a block scale overflows binary16    */
@@ -61,11 +70,12 @@ extern "C" {
 #define WOQ_PATH_FP32     1  /* FP32 products and accumulation (CUDA cores), exact codes      */
 #define WOQ_PATH_BF16_TC  2  /* tcgen05 tensor cores on bf16(X) and bf16(scale*code)          */
 #define WOQ_PATH_SPLIT_TC 3  /* tcgen05 tensor cores, FP32-accurate: X and scale*code each as  */
-                             /* bf16 hi + bf16 lo, all four products accumulated in FP32      */
+                             /* bf16 hi + bf16 lo, three products (lo*lo, below 2^-16 of each */
+                             /* term, dropped) accumulated in FP32                            */
 
 /*
  * One packed weight [n, k] in device memory.
- *   bits    4 or 8
+ *   bits    4, 5 or 8 (5: k % 128 == 0)
  *   block   must be 32
  *   n, k    rows (out features) and columns (in features); k % 32 == 0
  *   packed  device pointer, 64-byte aligned, n*k*bits/8 bytes in the layout above
@@ -102,9 +112,12 @@ int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, u
  * "How we built it": the separate GEMV path for decode). FP32 accuracy: within a 32-block
  * the codes are multiplied exactly and the block sum is scaled once, in FP32 (CUDA-core and
  * WOQ_GEMV_SPLIT_TC forms), or x and s*q go to the tcgen05 tensor cores as bf16 hi + lo pairs
- * (WOQ_GEMV_SPLIT_GEMM). The kernel is chosen by shape, as measured on B200: m >= 24 on
- * narrow matrices and m >= 48 on wide ones (n / 128 >= SM count) take WOQ_GEMV_SPLIT_GEMM,
- * 8 <= m < 48 on wide matrices WOQ_GEMV_SPLIT_TC, every other call the CUDA-core form.
+ * (WOQ_GEMV_SPLIT_GEMM), or the codes and x's signed digits go to the integer tensor cores
+ * (WOQ_GEMV_INT8_TC). The kernel is chosen by shape, as measured on B200: on matrices wide
+ * enough that 128-row tiles cover every SM (n / 128 >= SM count), m <= 2 the CUDA-core form,
+ * 3 <= m <= 4 WOQ_GEMV_INT8_TC for int8 and WOQ_GEMV_SPLIT_TC for int4, up to m = 32
+ * WOQ_GEMV_SPLIT_TC, from m = 33 WOQ_GEMV_SPLIT_GEMM; on narrower matrices the CUDA-core form
+ * below m = 16 and WOQ_GEMV_SPLIT_GEMM from there; int5 always the CUDA-core form.
  * Deterministic: the same inputs give the same bits on every call.
  *   x  device, [m, k] float32 row-major, 16-byte aligned
  *   w  host pointer to the weight descriptor (read during the call only)
@@ -264,7 +277,8 @@ size_t qgemm_workspace_bytes(int64_t m, const woq_weight *w, int32_t path);
  *        the kernel converts X itself, and when K is split across CTAs those CTAs form one
  *        thread-block cluster that sums the partials in shared memory, in a fixed order.
  *   path WOQ_PATH_FP32: the same FP32 arithmetic as qgemv, for any m.
- *   path WOQ_PATH_AUTO: BF16_TC if m >= 128, SPLIT_TC if 24 <= m < 128, else FP32.
+ *   path WOQ_PATH_AUTO: BF16_TC if m >= 128, SPLIT_TC if 16 <= m < 128, else FP32 (int5:
+ *        always FP32).
  *   X  device, [m, k] float32 row-major, 16-byte aligned
  *   Y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
  *   workspace  device, 256-byte aligned, at least qgemm_workspace_bytes(m, w, path) bytes

@@ -223,6 +223,23 @@ def test_auto_routes_batched_decode_to_the_split_gemm():
     name, n, k = workloads.DECODER_PROJ[6]
     W = workloads.weight(n, k, seed=7)
     w, _, _ = packed_from_weight(W, 4)
-    for m, same_as in ((16, "cuda_core"), (24, "split_gemm"), (64, "split_gemm")):
+    for m, same_as in ((15, "cuda_core"), (16, "split_gemm"), (64, "split_gemm")):
         x = workloads.activations(m, k, seed=m).cuda()
         assert torch.equal(woq.qgemv(x, w), woq.qgemv(x, w, path=same_as)), (m, same_as)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_auto_routes_on_a_wide_matrix(bits):
+    """Rows enough for one 128-row tile per SM and more: the measured choice by m and width."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n, k = 128 * sms + 1000, 512
+    W = workloads.weight(n, k, seed=70 + bits)
+    w, p, s = packed_from_weight(W, bits)
+    mid = "int8_tc" if bits == 8 else "split_tc"
+    for m, same_as in ((2, "cuda_core"), (3, mid), (4, mid), (5, "split_tc"), (32, "split_tc"),
+                       (33, "split_gemm")):
+        x = workloads.activations(m, k, seed=m)
+        a = woq.qgemv(x.cuda(), w)
+        assert torch.equal(a, woq.qgemv(x.cuda(), w, path=same_as)), (m, same_as)
+        rows = np.concatenate([np.random.default_rng(m).choice(n, 256, replace=False), [n - 1]])
+        assert max_rel(a.cpu().numpy()[:, rows], ref_rows(x.numpy(), p, s, bits, rows)) <= FP32_TOL

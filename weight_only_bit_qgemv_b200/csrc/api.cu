@@ -67,13 +67,18 @@ using woq::DevInfo;
 
 extern "C" {
 
-// qgemv's automatic choice, measured on B200. The tcgen05 split GEMM (no workspace) from
-// kGemmMinM rows on for the decoder projections and from kGemmMinMWide on for matrices wide
-// enough that 128-row tiles cover every SM (the lm_head); the small-batch mma.sync form for
-// the wide ones from kTcMinM rows up to there; the CUDA-core kernel otherwise.
-constexpr int64_t kTcMinM = 8;
-constexpr int64_t kGemmMinM = 24;
-constexpr int64_t kGemmMinMWide = 48;
+// qgemv's automatic choice, measured on B200 (graphs of calls over L2-cold copies). Matrices
+// wide enough that 128-row tiles cover every SM (the lm_head): the CUDA-core kernel for
+// m <= 2; for 3 <= m <= 4 the integer tensor cores (int8: 63.5 / 71.0 us against 77.1 on the
+// CUDA cores) or the small-batch mma.sync form (int4: 60.8 us against 94.9); the mma.sync form
+// up to m = 32 (int8 80-115 us, int4 61-109 us, where the tcgen05 split GEMM takes 146-164);
+// the split GEMM from m = 33 (at m = 47: 173 us against 272). Narrower matrices (the decoder's
+// projections): the CUDA-core kernel below m = 16, the split GEMM from there (m = 16: qkv 10.1
+// us against 11.8, down 11.2 against 12.05). int5 always takes the CUDA-core kernel.
+constexpr int64_t kTcMinMWide = 3;
+constexpr int64_t kI8TcMaxMWide = 4;
+constexpr int64_t kGemmMinM = 16;
+constexpr int64_t kGemmMinMWide = 33;
 
 int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t path,
                void *stream) {
@@ -104,7 +109,11 @@ int qgemv_path(const float *x, int64_t m, const woq_weight *w, float *y, int32_t
     const woq::GemmPlan plan = woq::plan_gemm_tc(m, w->n, w->k, dev.sm_count, SIZE_MAX, true);
     return woq::launch_gemm_tc(x, m, *w, y, nullptr, plan, s, dev);
   }
-  const bool tc = path == WOQ_GEMV_SPLIT_TC || (path == WOQ_GEMV_AUTO && m >= kTcMinM && wide);
+  if (path == WOQ_GEMV_AUTO && wide && w->bits == 8 && m >= kTcMinMWide && m <= kI8TcMaxMWide) {
+    rc = woq::launch_gemv_i8tc(x, m, *w, y, s, dev);
+    if (rc != 1) return rc;  // shapes it does not take go on below
+  }
+  const bool tc = path == WOQ_GEMV_SPLIT_TC || (path == WOQ_GEMV_AUTO && m >= kTcMinMWide && wide);
   if (tc) {
     rc = woq::launch_gemv_tc(x, m, *w, y, s, dev);
     if (rc != 1) return rc;
@@ -209,9 +218,9 @@ static int plan_sm_count() {
 
 // qgemm's automatic choice: the bf16 tensor-core GEMM for prefill-sized m, the FP32-accurate
 // split tensor-core GEMM for batched decode from kSplitMinM rows on (measured on B200 over
-// the decoder projections: faster than the CUDA-core kernel from there on), and the CUDA-core
-// kernel below that.
-constexpr int64_t kSplitMinM = 24;
+// the decoder projections and the lm_head: faster than the CUDA-core kernel from there on),
+// and the CUDA-core kernel below that.
+constexpr int64_t kSplitMinM = 16;
 
 static int resolve_path(int32_t path, int64_t m, int32_t bits) {
   if (path == WOQ_PATH_AUTO) {
