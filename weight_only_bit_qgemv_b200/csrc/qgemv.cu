@@ -298,9 +298,15 @@ constexpr int kEpiWrite = 0, kEpiArgmax = 1, kEpiSwiglu = 2, kEpiResidual = 3;
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// Registers for two CTAs per SM: the 17 warps of a 16-warp CTA need <= 56 (the launch bound);
+// the 9 warps of an 8-warp CTA need <= 96, as a sub-partition holding five of the 18 warps has
+// 16384 registers. The single-x-row 8-warp forms are held to 96 (the int4 lm_head form used
+// 100, which left one CTA per SM); forms with more x rows keep what they use, one CTA per SM.
+__host__ __device__ constexpr int bulk_max_regs(int nw, int mt) { return nw == 8 && mt == 1 ? 96 : 255; }
+
 // y carries no __restrict__: in residual mode `resid` may be y itself.
 template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
-__global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1)
+__global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1) __maxnreg__(bulk_max_regs(NW, MT))
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
                      const uint16_t *__restrict__ scales, float *y, int m, int n,
                      int k, int stages, int stage_bytes, int x_bytes,
