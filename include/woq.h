@@ -96,7 +96,7 @@ typedef struct woq_weight {
  * the soniqo Russian guide, "Implementation notes" (symmetric INT8 block-32). For each row
  * r and block j:
  *   a = max |W[r, 32j .. 32j+31]|                                  (exact, over the floats)
- *   s = binary16 round-half-even of (double)a / qmax, qmax = 7 (int4) or 127 (int8)
+ *   s = binary16 round-half-even of (double)a / qmax, qmax = 7 (int4), 15 (int5) or 127 (int8)
  *   q = clamp(round-half-even((double)w / (double)s), -2^(bits-1), 2^(bits-1)-1), or 0 if s == 0
  * and writes q into `packed` and the bit pattern of s into `scales`, in the layout above.
  *   W       [n, k] float32, row-major
@@ -118,7 +118,10 @@ int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, u
  * 3 <= m <= 4 WOQ_GEMV_INT8_TC for int8 and WOQ_GEMV_SPLIT_TC for int4, up to m = 32
  * WOQ_GEMV_SPLIT_TC, from m = 33 WOQ_GEMV_SPLIT_GEMM; on narrower matrices the CUDA-core form
  * below m = 16 and WOQ_GEMV_SPLIT_GEMM from there; int5 always the CUDA-core form.
- * Deterministic: the same inputs give the same bits on every call.
+ * Deterministic: the same inputs give the same bits on every call. For int5 at m = 1 the
+ * CUDA-core form may split each row's k (k > 1024) across 2 or 4 warps and add their sums
+ * in a fixed order, so such a row can differ in the last bits from the same row computed in
+ * a batch; at one m, qgemv, qgemv_argmax and qgemv_residual add in the same order.
  *   x  device, [m, k] float32 row-major, 16-byte aligned
  *   w  host pointer to the weight descriptor (read during the call only)
  *   y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten

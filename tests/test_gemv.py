@@ -184,6 +184,24 @@ def test_small_batch_tensor_core_ragged_rows(m):
     assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, 4)) <= FP32_TOL
 
 
+@pytest.mark.parametrize("bits", [4, 5, 8])
+@pytest.mark.parametrize("n,k", [(1024, 2048), (1024, 3072), (1001, 2048), (999, 3072), (5, 4096),
+                                 (300, 8192)])
+def test_split_k_inside_the_cta(bits, n, k):
+    """m = 1 over rows of more than 32 blocks: for int5 the 16-warp launch splits each row's K
+    across 2 or 4 warps and adds their partial sums in a fixed order (int4 and int8 run the
+    same shapes unsplit); ragged last tiles are read from global memory, and a matrix of fewer
+    rows than one split tile takes the unsplit form."""
+    W = workloads.weight(n, k, seed=n + k + bits)
+    w, p, s = packed_from_weight(W, bits)
+    x = workloads.activations(1, k, seed=k)
+    buf, y = guarded_out(1, n)
+    woq.qgemv(x.cuda(), w, out=y)
+    assert tail_intact(buf, 1, n)
+    assert torch.equal(y, woq.qgemv(x.cuda(), w))
+    assert max_rel(y.cpu().numpy(), ref_rows(x.numpy(), p, s, bits)) <= FP32_TOL
+
+
 def test_split_tc_rejects_shapes_outside_its_limits():
     w, _, _ = packed_raw(256, 96, 8, seed=5)  # k % 256 != 0
     x = workloads.activations(4, 96, seed=1).cuda()

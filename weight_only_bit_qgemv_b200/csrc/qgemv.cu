@@ -38,17 +38,18 @@ using namespace gemv;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
-// Dot products of RW consecutive weight rows with MT staged x rows, lane l taking blocks
-// l, l+32, ... . SMEM: rows come from a shared-memory stage (all RW rows present);
+// Dot products of RW consecutive weight rows with MT staged x rows over blocks [b0, b1) of
+// each row, lane l taking blocks b0+l, b0+l+32, ... . SMEM: rows come from a shared-memory stage (all RW rows present);
 // otherwise from global memory, rows at or past `valid` reading as zero.
 template <int BITS, int MT, int RW, bool SMEM>
 __device__ __forceinline__ void rows_dot(const float4 *__restrict__ xs4, int units_row, int spr,
                                          int lane, const uint8_t *codes, size_t row_stride,
-                                         const uint16_t *scs, int valid, float (&acc)[RW][MT]) {
+                                         const uint16_t *scs, int valid, float (&acc)[RW][MT],
+                                         int b0, int b1) {
   if constexpr (BITS == 5) {
     // int5: a block's 16 bytes of low nibbles at 16 b, its high-bit word at k/2 + 4 b
     const int half = spr * 16;
-    for (int b = lane; b < spr; b += 32) {
+    for (int b = b0 + lane; b < b1; b += 32) {
       uint4 lo[RW];
       uint32_t hw[RW];
       float sc[RW];
@@ -75,7 +76,7 @@ __device__ __forceinline__ void rows_dot(const float4 *__restrict__ xs4, int uni
     }
   } else {
   constexpr int kBlockBytes = BITS * 4;  // 16 (int4) or 32 (int8)
-  for (int b = lane; b < spr; b += 32) {
+  for (int b = b0 + lane; b < b1; b += 32) {
     uint4 lo[RW], hi[RW];
     float sc[RW];
 #pragma unroll
@@ -271,6 +272,7 @@ struct BulkShared {
   uint64_t empty[kMaxStages];
   unsigned long long amax[8];  // argmax mode: this CTA's best key per activation row
   int abort;
+  int stop[2];  // split-K: a compute warp's stage wait gave up on a tile of this parity
 };
 static_assert(sizeof(BulkShared) <= kBulkHeader, "header too small");
 
@@ -305,16 +307,27 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 __host__ __device__ constexpr int bulk_max_regs(int nw, int mt) { return nw == 8 && mt == 1 ? 96 : 255; }
 
 // y carries no __restrict__: in residual mode `resid` may be y itself.
-template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
+//
+// KS > 1 (split-K inside the CTA, one x row, any epilogue but SwiGLU): the KS consecutive
+// warps of a group share the group's RW rows, warp part p taking blocks
+// [p * spr / KS, (p + 1) * spr / KS) of each row. After each tile every warp leaves its
+// reduced partial sums in shared memory (two buffers, by tile parity), the compute warps meet
+// at a barrier, and the group's first warp adds the KS partials in part order, so the result
+// does not depend on timing. The barrier is reached by every compute warp on every tile: a
+// warp whose stage wait gave up skips the arithmetic and raises the tile's stop flag, and
+// all compute warps leave the loop together after that tile's barrier.
+template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite, int KS = 1>
 __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1) __maxnreg__(bulk_max_regs(NW, MT))
     gemv_bulk_kernel(const float *__restrict__ x, const uint8_t *__restrict__ packed,
                      const uint16_t *__restrict__ scales, float *y, int m, int n,
                      int k, int stages, int stage_bytes, int x_bytes,
                      unsigned long long *__restrict__ keys = nullptr, const float *resid = nullptr) {
   constexpr int kBulkWarps = NW;
-  constexpr int TR = kBulkWarps * RW;
+  constexpr int TR = kBulkWarps / KS * RW;
   constexpr bool AMAX = EPI == kEpiArgmax;
   static_assert(EPI != kEpiSwiglu || RW % 2 == 0, "gate/up pairs need an even row count");
+  static_assert(KS == 1 || (MT == 1 && NW % KS == 0 && EPI != kEpiSwiglu),
+                "split-K takes one x row and the plain, residual or argmax epilogue");
   extern __shared__ __align__(128) uint8_t smem[];
   BulkShared &sh = *reinterpret_cast<BulkShared *>(smem);
   float4 *xs4 = reinterpret_cast<float4 *>(smem + kBulkHeader);
@@ -339,6 +352,7 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1) __maxnreg_
       ptx::mbar_init(&sh.empty[s], kBulkWarps);
     }
     sh.abort = 0;
+    sh.stop[0] = sh.stop[1] = 0;
     for (int mm = 0; mm < MT; ++mm) sh.amax[mm] = 0ull;
     ptx::fence_mbar_init();
   }
@@ -398,27 +412,33 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1) __maxnreg_
   ptx::pdl_launch_dependents();
   unsigned long long best = 0ull;  // argmax mode: this lane's best key (activation row lane % MT)
 
+  const int part = warp % KS;  // split-K: this warp's share of each row's blocks
+  const int b0 = part * (spr / KS), b1 = KS == 1 ? spr : b0 + spr / KS;
+  float *pbuf = reinterpret_cast<float *>(ring + static_cast<size_t>(stages) * stage_bytes);
+
   for (int tile = blockIdx.x, i = 0; tile < num_tiles; tile += gridDim.x, ++i) {
     const bool staged = tile < full_tiles;
     const int s = i % stages;
     // The outcome is made warp-uniform: shuffles and the elected arrival follow.
     // Bandwidth-bound launches (NW = 8) let waiting warps sleep so that the computing ones
     // get the issue slots; latency-bound ones (NW = 16) poll.
-    if (staged && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.full[s], (i / stages) & 1,
-                                                                   kGemvWaitLimit, abort,
-                                                                   NW == 8 ? 1000u : 0u))) {
+    const bool ok = !staged || __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sh.full[s], (i / stages) & 1,
+                                                                              kGemvWaitLimit, abort,
+                                                                              NW == 8 ? 1000u : 0u));
+    if (!ok) {
       gemv_record_timeout(abort);
-      break;
+      if constexpr (KS == 1) break;
+      sh.stop[i & 1] = 1;  // written only by compute warps, read by all after this tile's barrier
     }
     const uint8_t *stage = ring + static_cast<size_t>(s) * stage_bytes;
-    const int lrow0 = warp * RW;  // this warp's first row within the tile
+    const int lrow0 = warp / KS * RW;  // this warp's first row within the tile
     const int row0 = tile * TR + lrow0;
     // Residual mode: the lane that will store output (row0 + lane / MT, x row lane % MT)
     // fetches its residual now, so that the load's latency hides behind the dot products.
     float res = 0.f;
     if constexpr (EPI == kEpiResidual) {
       const int rr = lane / MT, mm = lane % MT;
-      if (rr < RW && row0 + rr < n && m0 + mm < m)
+      if (part == 0 && rr < RW && row0 + rr < n && m0 + mm < m)
         res = resid[static_cast<size_t>(m0 + mm) * n + row0 + rr];
     }
     float acc[RW][MT];
@@ -427,16 +447,16 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1) __maxnreg_
 #pragma unroll
       for (int mm = 0; mm < MT; ++mm) acc[r][mm] = 0.f;
 
-    if (staged) {
+    if (staged && ok) {
       rows_dot<BITS, MT, RW, true>(xs4, units_row, spr, lane, stage + lrow0 * row_bytes, row_bytes,
                                    reinterpret_cast<const uint16_t *>(stage + code_bytes) + lrow0 * spr,
-                                   RW, acc);
-    } else {
+                                   RW, acc, b0, b1);
+    } else if (!staged) {
       rows_dot<BITS, MT, RW, false>(xs4, units_row, spr, lane,
                                     packed + static_cast<size_t>(row0) * row_bytes, row_bytes,
-                                    scales + static_cast<size_t>(row0) * spr, n - row0, acc);
+                                    scales + static_cast<size_t>(row0) * spr, n - row0, acc, b0, b1);
     }
-    if (staged) {
+    if (staged && ok) {
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&sh.empty[s]);
     }
@@ -452,6 +472,27 @@ __global__ void __launch_bounds__(bulk_threads(NW), NW == 16 ? 2 : 1) __maxnreg_
         v += __shfl_xor_sync(0xffffffffu, v, 1);
         acc[r][mm] = v;
       }
+    if constexpr (KS > 1) {
+      float *pb = pbuf + (i & 1) * (kBulkWarps * RW);
+      if (lane < RW) {
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+          if (lane == r) pb[warp * RW + r] = acc[r][0];
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kBulkWarps * 32) : "memory");
+      // Every compute warp reads the same flag after the same barrier, so all leave together;
+      // the next tile's flag is the other one, so a warp already on that tile cannot change
+      // this outcome for a warp still reading it.
+      if (*static_cast<volatile int *>(&sh.stop[i & 1])) break;
+      if (part != 0) continue;
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        float v = pb[warp * RW + r];
+#pragma unroll
+        for (int p = 1; p < KS; ++p) v += pb[(warp + p) * RW + r];
+        acc[r][0] = v;
+      }
+    }
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
@@ -599,22 +640,24 @@ constexpr size_t kStageTarget = 20 * 1024;   // bytes per ring stage to aim for
 constexpr size_t kStageTargetWide = 36 * 1024;
 constexpr size_t kCtaSmemBudget = 100 * 1024;  // so that two CTAs fit on an SM
 
-template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite>
+template <int BITS, int MT, int RW, int NW, int EPI = kEpiWrite, int KS = 1>
 int launch_bulk_t(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
                   const DevInfo &dev, bool pdl, size_t stage_bytes, size_t x_bytes,
                   unsigned long long *keys = nullptr, const float *resid = nullptr) {
-  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW, EPI>;
+  auto kern = gemv_bulk_kernel<BITS, MT, RW, NW, EPI, KS>;
   constexpr int kBulkThreads = bulk_threads(NW);
-  constexpr int TR = NW * RW;
+  constexpr int TR = NW / KS * RW;
+  constexpr size_t kPartialBytes = KS > 1 ? 2 * NW * RW * sizeof(float) : 0;
   const int64_t num_tiles = (w.n + TR - 1) / TR;
   const int64_t full_tiles = w.n / TR;
   // stages: enough for the tiles one CTA will see, within the smem budget
   const int64_t want_grid = std::min<int64_t>(num_tiles, static_cast<int64_t>(dev.sm_count) * 2);
   int64_t stages = want_grid > 0 ? (full_tiles + want_grid - 1) / want_grid : 1;
-  const int64_t fit = (static_cast<int64_t>(kCtaSmemBudget) - kBulkHeader - static_cast<int64_t>(x_bytes)) /
+  const int64_t fit = (static_cast<int64_t>(kCtaSmemBudget) - kBulkHeader - static_cast<int64_t>(x_bytes) -
+                       static_cast<int64_t>(kPartialBytes)) /
                       static_cast<int64_t>(stage_bytes);
   stages = std::max<int64_t>(1, std::min<int64_t>({stages, fit, kMaxStages}));
-  const size_t smem = kBulkHeader + x_bytes + stages * stage_bytes;
+  const size_t smem = kBulkHeader + x_bytes + stages * stage_bytes + kPartialBytes;
   const int nb = blocks_per_sm(reinterpret_cast<const void *>(kern), smem, dev, kBulkThreads,
                                kCtaSmemBudget);
   if (nb <= 0) return WOQ_ECUDA;
@@ -676,12 +719,55 @@ int launch_bulk_nw(const float *x, int64_t m, const woq_weight &w, float *y, cud
                                               x_bytes, keys, resid);
 }
 
+// Split-K for the 16-warp launch of an int5 call with one x row (m == 1): while a warp's share
+// of a row is more than one block per lane, halve it (up to 4 parts), as long as the CTAs
+// still number at most two per SM and the scale ranges of a tile stay 16-byte multiples.
+// Returns 1 when it does not split.
+//
+// Measured on B200 over the decoder block (four dependent launches, programmatic dependent
+// launch): int5 11 % faster per step (15.7 -> 14.0 us), its unpack being the heaviest; int4
+// 19 % slower (11.0 -> 13.2 us) even though o and down alone each got 0.1 us faster, because
+// the split launches' extra CTAs leave no room on the SMs for the next launch's CTAs to start
+// streaming their weights early. So int4 and int8 do not split.
+//
+// Calls with m > 1 never split, also where their x rows go one at a time, so that qgemv,
+// qgemv_argmax and qgemv_residual at the same m add a row's products in the same order
+// (bitwise the same outputs); an int5 row at m = 1 may differ in the last bits from the same
+// row in a batch.
+inline int bulk_splits(const woq_weight &w, int64_t m, int sms) {
+  if (m != 1 || w.bits != 5) return 1;
+  const int64_t spr = w.k / 32;
+  int ks = 1;
+  while (ks < 4 && spr / ks > 32 && spr % (2 * ks) == 0 && w.n / (16 / (2 * ks)) <= 2 * static_cast<int64_t>(sms) &&
+         w.n >= 16 / (2 * ks))
+    ks *= 2;
+  return ks;
+}
+
+template <int BITS, int EPI>
+int launch_bulk_split(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
+                      const DevInfo &dev, bool pdl, size_t row_total, size_t x_bytes, int ks,
+                      const float *resid = nullptr, unsigned long long *keys = nullptr) {
+  const size_t stage_bytes = (static_cast<size_t>(16 / ks) * row_total + 127) & ~size_t(127);
+  if (kBulkHeader + x_bytes + stage_bytes + 2 * 16 * sizeof(float) > kCtaSmemBudget) return 1;
+  if (ks == 2)
+    return launch_bulk_t<BITS, 1, 1, 16, EPI, 2>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys, resid);
+  if (ks == 4)
+    return launch_bulk_t<BITS, 1, 1, 16, EPI, 4>(x, m, w, y, s, dev, pdl, stage_bytes, x_bytes, keys, resid);
+  return 1;
+}
+
 template <int BITS, int MT>
 int try_bulk(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream_t s,
              const DevInfo &dev, bool pdl) {
   const size_t row_total = static_cast<size_t>(w.k) * BITS / 8 + static_cast<size_t>(w.k) / 16;
   const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
   if constexpr (MT == 1) {
+    const int ks = bulk_splits(w, m, dev.sm_count);
+    if (ks > 1) {
+      const int rc = launch_bulk_split<BITS, kEpiWrite>(x, m, w, y, s, dev, pdl, row_total, x_bytes, ks);
+      if (rc != 1) return rc;
+    }
     // 16 warps where each CTA of the grid gets at most two tiles (latency-bound launches).
     const int rw16 = bulk_rows_per_warp(16, 2, row_total);
     const int64_t tiles16 = w.n / (16 * rw16);
@@ -789,6 +875,15 @@ int argmax_bulk(const float *x, int64_t m, const woq_weight &w, unsigned long lo
   return with_fitting_mt(m, [&](auto mt_tag) -> int {
     constexpr int MT = decltype(mt_tag)::value;
     const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
+    if constexpr (MT == 1) {
+      // where qgemv splits K, the pick does too, so that it sees the same output bits
+      const int ks = bulk_splits(w, m, dev.sm_count);
+      if (ks > 1) {
+        const int rc = launch_bulk_split<BITS, kEpiArgmax>(x, m, w, nullptr, s, dev, true, row_total, x_bytes,
+                                                           ks, nullptr, keys);
+        if (rc != 1) return rc;
+      }
+    }
     return launch_bulk_nw<BITS, MT, 8, kEpiArgmax>(x, m, w, nullptr, s, dev, true, row_total, x_bytes, keys);
   });
 }
@@ -802,6 +897,12 @@ int residual_bulk(const float *x, int64_t m, const woq_weight &w, const float *r
     constexpr int MT = decltype(mt_tag)::value;
     const size_t x_bytes = (static_cast<size_t>(MT) * w.k * sizeof(float) + 127) & ~size_t(127);
     if constexpr (MT == 1) {
+      const int ks = bulk_splits(w, m, dev.sm_count);
+      if (ks > 1) {
+        const int rc = launch_bulk_split<BITS, kEpiResidual>(x, m, w, y, s, dev, true, row_total, x_bytes,
+                                                             ks, r);
+        if (rc != 1) return rc;
+      }
       const int rw16 = bulk_rows_per_warp(16, 2, row_total);
       const int64_t tiles16 = w.n / (16 * rw16);
       if (tiles16 >= 1 && tiles16 <= 2 * static_cast<int64_t>(dev.sm_count)) {
