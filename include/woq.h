@@ -125,7 +125,9 @@ int qpack(const float *W, int64_t n, int64_t k, int32_t bits, uint8_t *packed, u
  *   x  device, [m, k] float32 row-major, 16-byte aligned
  *   w  host pointer to the weight descriptor (read during the call only)
  *   y  device, [m, n] float32 row-major, 16-byte aligned; fully overwritten
- * Limits: k <= 32768 (the x rows are staged in shared memory). Errors: WOQ_EINVAL,
+ * Limits: k <= 32768 (the x rows are staged in shared memory); int5 k <= 10752 (its only
+ * kernel stages one x row beside a stage of 8 weight rows in 100 KB; at m = 1 over few rows
+ * a 4-row split-K stage can take somewhat more). Errors: WOQ_EINVAL,
  * WOQ_ESHAPE, WOQ_EALIGN, WOQ_EDEVICE, WOQ_ECUDA.
  */
 int qgemv(const float *x, int64_t m, const woq_weight *w, float *y, void *stream);
@@ -235,7 +237,10 @@ int qgemv_argmax(const float *x, int64_t m, const woq_weight *w, int64_t *idx, f
  *             must be zero before the first call; every call that returns WOQ_OK leaves them
  *             zero again (after a WOQ_ETIMEOUT from woq_device_status, zero them before reuse).
  *             Calls sharing one workspace must be ordered on one stream.
- * Each item: w as for qgemv with k % 256 == 0 and k <= 8192; x [m, k] and y device, 16-byte
+ * Each item: w as for qgemv with k % 256 == 0 and k <= 8192 (the x rows, m rounded up to 1,
+ * 2, 4 or 8 of them at the largest k, are staged in each CTA's shared memory beside at least
+ * two weight stages: every k fits at m <= 4, at m = 8 up to about 5600; WOQ_ESHAPE beyond);
+ * x [m, k] and y device, 16-byte
  * aligned, y not overlapping x; r (WOQ_EPI_RESIDUAL only) device, 16-byte aligned, equal to y
  * or not overlapping it. Errors: WOQ_EINVAL, WOQ_ESHAPE, WOQ_EALIGN, WOQ_EWORKSPACE,
  * WOQ_EDEVICE, WOQ_ECUDA. The launch holds one CTA per SM, and its CTAs wait for one another

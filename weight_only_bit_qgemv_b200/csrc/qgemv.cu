@@ -787,15 +787,23 @@ int pick_mt(const float *x, int64_t m, const woq_weight &w, float *y, cudaStream
   while (mt > 1 && static_cast<size_t>(mt) * w.k * sizeof(float) > limit) mt /= 2;
   if (static_cast<size_t>(mt) * w.k * sizeof(float) > limit) return WOQ_ESHAPE;
   int rc = 1;
-  switch (mt) {
-    case 1: rc = try_bulk<BITS, 1>(x, m, w, y, s, dev, pdl); break;
-    case 2: rc = try_bulk<BITS, 2>(x, m, w, y, s, dev, pdl); break;
-    case 4: rc = try_bulk<BITS, 4>(x, m, w, y, s, dev, pdl); break;
-    default: rc = try_bulk<BITS, 8>(x, m, w, y, s, dev, pdl); break;
-  }
+  auto bulk = [&](int t) {
+    switch (t) {
+      case 1: return try_bulk<BITS, 1>(x, m, w, y, s, dev, pdl);
+      case 2: return try_bulk<BITS, 2>(x, m, w, y, s, dev, pdl);
+      case 4: return try_bulk<BITS, 4>(x, m, w, y, s, dev, pdl);
+      default: return try_bulk<BITS, 8>(x, m, w, y, s, dev, pdl);
+    }
+  };
+  rc = bulk(mt);
   if (rc != 1) return rc;
   if constexpr (BITS == 5) {
-    return WOQ_ESHAPE;  // int5: the staged kernel only
+    // int5 has the staged kernel only: fewer x rows per CTA until they fit beside a stage
+    for (int t = mt / 2; t >= 1; t /= 2) {
+      rc = bulk(t);
+      if (rc != 1) return rc;
+    }
+    return WOQ_ESHAPE;
   } else {
     switch (mt) {
       case 1: return pick_ru<BITS, 1>(x, m, w, y, s, dev, pdl);
