@@ -791,7 +791,7 @@ def run_prefill(layers, groups, device, m: int, peaks, peak_kind, stream, world,
 def run_batched_decode(layers, groups, device, m: int, peaks, peak_kind, stream, world, flush,
                        lm_head=None):
     """Batched decode: m activation rows through every fused projection of every block via
-    qgemm's automatic path (the FP32-accurate split tensor-core GEMM for 24 <= m < 128), then
+    qgemm's automatic path (the FP32-accurate split tensor-core GEMM for 16 <= m < 128), then
     the int8 lm_head if given. One decoder step = 28 blocks (+ lm_head), replayed from a CUDA
     graph after an L2 flush, median of 3."""
     import weight_only_bit_qgemv_b200 as woq
@@ -814,7 +814,7 @@ def run_batched_decode(layers, groups, device, m: int, peaks, peak_kind, stream,
     us_block = ms_blocks * 1e3 / len(layers)
     step_bytes = decode_step_bytes(layers[0])
     block_gbs = step_bytes / (us_block * 1e-6) / 1e9
-    path = "split_tc" if 24 <= m < 128 else ("bf16_tc" if m >= 128 else "fp32")
+    path = "split_tc" if 16 <= m < 128 else ("bf16_tc" if m >= 128 else "fp32")
     out = {"workload": f"decoder_m{m}" + ("_plus_lm_head" if lm_head is not None else ""),
            "dtype": "f32 (split tensor-core form: bf16 hi+lo operands, f32 accumulate)"
                     if path == "split_tc" else "f32",
