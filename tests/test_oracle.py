@@ -225,6 +225,25 @@ def test_int5_high_bit_positions(e, bit):
     assert word == 1 << bit
 
 
+@pytest.mark.parametrize("e,bit", [(0, 0), (3, 12), (4, 16), (8, 1), (29, 23), (31, 31)])
+def test_int5_high_bit_position_function(e, bit):
+    """The position function itself, on the hand-derived table above (element e of a block:
+    bit e/8 + 4(e%4) + 16((e%8)/4) of the high-bit word)."""
+    assert oracle.int5_high_bit_position(e) == bit
+
+
+def test_int5_high_bit_positions_cover_the_word_once():
+    assert sorted(oracle.int5_high_bit_position(e) for e in range(32)) == list(range(32))
+
+
+@pytest.mark.parametrize("bits,K,expect", [(4, 1024, 512), (5, 1024, 640), (8, 1024, 1024),
+                                           (4, 32, 16), (5, 128, 80), (8, 96, 96)])
+def test_row_bytes_is_the_packed_row_length(bits, K, expect):
+    assert oracle.row_bytes(K, bits) == expect
+    q = np.zeros((3, K), dtype=np.int32)
+    assert oracle.pack(q, bits).shape == (3, expect)
+
+
 # ---------------------------------------------------------------------------
 # special matrices, invariants, linearity, error bound
 # ---------------------------------------------------------------------------
