@@ -1043,6 +1043,17 @@ def cpu_legs(groups, layer0_gpu, xs_gpu):
         lambda: oracle.qgemv_ref(x3, *pk3), pk3[0].nbytes + pk3[1].nbytes, "GB/s", 1e9,
         f"rows 0..{rows - 1} of the int8 lm_head [151936x1024] at M=1 (the rate is per byte, "
         "so it stands for the whole matrix)")
+    # the same lm_head sample as int4 and int5, and decoder block 0 as int5
+    for bits in (4, 5):
+        pkb = oracle_pack(W, bits)
+        legs[f"lm_head_m1_int{bits}"], _ = cpu_baseline(
+            lambda pkb=pkb: oracle.qgemv_ref(x3, *pkb), pkb[0].nbytes + pkb[1].nbytes, "GB/s", 1e9,
+            f"rows 0..{rows - 1} of the int{bits} lm_head [151936x1024] at M=1 (the rate is per "
+            "byte, so it stands for the whole matrix)")
+    packed5, xs5 = oracle_layer_inputs(groups, bits=5)
+    legs["decoder_block_m1_int5"], _ = cpu_baseline(
+        lambda: oracle_decode_pass(packed5, xs5), sum(pk.nbytes + sc.nbytes for pk, sc, _ in packed5),
+        "GB/s", 1e9, "decoder block 0 (7 projections, M=1, int5) through the NumPy float64 oracle")
     # configuration 4: prefill M=512, block 0's 7 projections (1/28 of a pass)
     packed512, xs512 = oracle_layer_inputs(groups, m=512)
     legs["prefill_m512"], _ = cpu_baseline(
@@ -1220,6 +1231,8 @@ def main(argv=None):
             out["parity_chain"] = chain_parity(chain_step, oracle_chain_block0())
         configs["decoder_block_m1"]["cpu_baseline"] = out["cpu_baseline"]
         key_of = {"single_qgemv_m1": "single_qgemv_m1", "lm_head_m1_int8": "lm_head_m1_int8",
+                  "lm_head_m1_int4": "lm_head_m1_int4", "lm_head_m1_int5": "lm_head_m1_int5",
+                  "decoder_block_m1_int5": "decoder_block_m1_int5",
                   "prefill_m512": "prefill_m512", "decoder_m64": "decoder_m64_plus_lm_head",
                   "prefill_m4096": "prefill_m4096_plus_lm_head"}
         for leg, cfg in key_of.items():
