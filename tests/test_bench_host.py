@@ -81,3 +81,21 @@ def test_committed_traffic_file_parses():
     for workload in ("decoder_block_m1", "lm_head_m1_int8"):
         v = bench.measured_traffic(workload)
         assert v is None or v > 0
+
+
+def test_reference_arm_prints_the_contract_line_on_rank_zero_only():
+    """`bench.py --impl reference`: the oracle on host cores, a bounded sample per step, the
+    same metric and config as the GPU arm, zero copy bytes; other ranks print nothing."""
+    import types
+
+    import bench
+
+    args = types.SimpleNamespace(steps=2, warmup=3)
+    assert bench.run_reference(args, world=2, rank=1, budget_s=1.0) is None
+    out = bench.run_reference(args, world=1, rank=0, budget_s=1.0)
+    assert out["impl"] == "reference" and out["metric"] == bench.METRIC
+    assert out["unit"] == "GB/s" and out["value"] > 0 and out["steps"] == 2 and out["warmup"] == 3
+    assert out["config"]["workload"] == "decoder_block_m1"
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
+    assert out["e2e"] == {"value": out["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
