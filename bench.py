@@ -1,6 +1,7 @@
 """Benchmark of the weight-only block-32 qgemv/qgemm path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--legs chain,int5,single,lm_head,prefill,batched,epilogues,cpu]
 
 Headline workload ("decoder_block_m1"): one Qwen3-0.6B-style decoder block at decode, M = 1,
 int4 block-32 weights: the 7 projections q[2048x1024], k[1024x1024], v[1024x1024],
@@ -23,7 +24,10 @@ every step), `roofline` (the decode kernel against the measured HBM copy bandwid
 `parity` (GPU vs oracle on the sampled step), and `configs`: one object per workload
 configuration of the benchmark (a single qgemv; the decoder block; the int8 lm_head; prefill
 M = 512 over all 28 blocks; batched decode M = 64 and prefill M = 4096 over all 28 blocks
-plus the lm_head), each with its own dtype, roofline and CPU baseline.
+plus the lm_head), each with its own dtype, roofline and CPU baseline, beside the decoder
+block as one `qgemv_chain` launch, the int4 and int5 lm_head, the int5 decoder block and the
+fused epilogues. `--legs` runs a subset (the headline always runs); each leg runs inside an
+NVTX range named after its workload, for `ncu --nvtx-include`.
 """
 
 from __future__ import annotations
