@@ -130,3 +130,22 @@ def test_binding_constants_match_the_header():
     assert len(defines) >= 17
     for name, value in defines.items():
         assert getattr(_lib, name) == int(value), name
+
+
+def test_python_binding_names_every_compute_call():
+    """The package exposes each compute call of the C ABI under the same name, and its
+    wrappers refuse host tensors before calling into the library."""
+    import pytest
+    import torch
+
+    import weight_only_bit_qgemv_b200 as woq
+
+    for name in ("qpack", "qgemv", "qgemv_swiglu", "qgemv_residual", "qgemv_argmax", "qgemv_chain",
+                 "qgemm", "qgemm_workspace_bytes", "qgemm_bf16_noalloc"):
+        assert name in woq.__all__ and callable(getattr(woq, name)), name
+    w = woq.PackedWeight(torch.zeros(4, 16, dtype=torch.uint8), torch.zeros(4, 1, dtype=torch.int16),
+                         4, 4, 32)
+    x = torch.zeros(1, 32)
+    for call in (woq.qgemv, woq.qgemv_swiglu, woq.qgemv_argmax, woq.qgemm, woq.qgemm_bf16_noalloc):
+        with pytest.raises(ValueError):
+            call(x, w)

@@ -45,6 +45,7 @@ __all__ = [
     "qgemv_chain",
     "qgemm",
     "qgemm_workspace_bytes",
+    "qgemm_bf16_noalloc",
     "device_status",
     "launch_count",
     "WoqError",
@@ -263,6 +264,23 @@ def qgemm(
         _lib.lib().qgemm(_ptr(X), m, ctypes.byref(d), _ptr(out), p, ws_ptr, ws_bytes, _stream(stream)),
         "qgemm",
     )
+    return out
+
+
+def qgemm_bf16_noalloc(X: torch.Tensor, w: PackedWeight, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """The bf16 tensor-core qgemm with no workspace and no device allocation in the library
+    (C ABI ``qgemm_bf16_noalloc``): the bf16 copy of X goes to a fixed 32 MiB scratch array
+    of the library's own, so m * k * 2 bytes must fit in it. ``out`` is allocated here by
+    PyTorch when it is not given."""
+    if X.dtype != torch.float32 or not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous 2-D float32 CUDA tensor")
+    m = X.shape[0]
+    if out is None:
+        out = torch.empty(m, w.n, dtype=torch.float32, device=X.device)
+    d = w.desc()
+    _lib.check(_lib.lib().qgemm_bf16_noalloc(_ptr(X), m, ctypes.byref(d), _ptr(out), _stream(stream)),
+               "qgemm_bf16_noalloc")
     return out
 
 
